@@ -1,0 +1,184 @@
+"""Seeded synthetic inputs for the fused-MoE layer.
+
+This module is the one piece shared by the CUDA path's tests/benchmark and the
+CPU oracle: it draws the inputs and nothing else.  It holds none of the layer's
+arithmetic (no routing, permutation, GEMM, activation or combine).  Weights
+that are stored in FP8 are prepared here the way a checkpoint would be (one
+fp32 scale per expert matrix, scale = amax / 448); that is input preparation,
+not a step of the layer.
+
+Every tensor comes from its own Philox stream keyed by (seed, tensor name,
+expert), so a tensor is the same bits whatever else is generated and however
+many threads generate it.  Everything is produced on the host as numpy arrays:
+bf16 tensors as uint16 bit patterns, FP8 E4M3 tensors as uint8 codes.
+
+Workloads (the layer shapes the library is measured and checked on):
+  tiny                 T=16  H=256  I=512   E=8   top-2 softmax, bf16
+  mixtral_decode       T=64 (1, 8) H=4096 I=14336 E=8 top-2 softmax, bf16
+  mixtral_prefill_fp8  T=4096 H=4096 I=14336 E=8 top-2 softmax, E4M3 weights and
+                       activations, static per-tensor scales
+  dsv3_decode_fp8w     T=1/8/32/128 H=7168 I=2048 E=256 top-8 sigmoid x2.5
+                       (renormalised) + 1 shared expert, E4M3 weights, bf16 acts
+  qwen2_skewed_prefill T=8192 H=2048 I=1408 E=60 top-4 softmax, bf16, router
+                       logits N(0,1) + Zipf(1.2) expert bias
+Distributions: x ~ N(0,1); router weight W_g ~ N(0, 0.02^2) in bf16 and
+logits = fp32(x . W_g^T) computed in double; expert weights ~ N(0, 1/fan_in)
+(standard deviation 1/sqrt(fan_in), fan_in = H for W1/W3 and I for W2).
+"""
+from __future__ import annotations
+
+import dataclasses
+import os
+import zlib
+from concurrent.futures import ThreadPoolExecutor
+
+import numpy as np
+import torch
+
+BF16, E4M3 = 0, 1
+SOFTMAX, SIGMOID = 0, 1
+E4M3_MAX = 448.0
+
+
+@dataclasses.dataclass(frozen=True)
+class Workload:
+    name: str
+    T: int
+    H: int
+    I: int
+    E: int
+    k: int
+    n_shared: int = 0
+    gate: int = SOFTMAX
+    renorm: bool = True
+    routed_scale: float = 1.0
+    wdtype: int = BF16
+    adtype: int = BF16
+    logits: str = "router"          # "router" (x . W_g) or "zipf" (N(0,1) + bias)
+    zipf_s: float = 1.2
+    seed: int = 0
+
+    @property
+    def E_tot(self) -> int:
+        return self.E + self.n_shared
+
+    def with_T(self, T: int) -> "Workload":
+        return dataclasses.replace(self, T=T)
+
+
+WORKLOADS = {
+    "tiny": Workload("tiny", T=16, H=256, I=512, E=8, k=2),
+    "mixtral_decode": Workload("mixtral_decode", T=64, H=4096, I=14336, E=8, k=2),
+    "mixtral_prefill_fp8": Workload("mixtral_prefill_fp8", T=4096, H=4096, I=14336, E=8, k=2,
+                                    wdtype=E4M3, adtype=E4M3),
+    "dsv3_decode_fp8w": Workload("dsv3_decode_fp8w", T=128, H=7168, I=2048, E=256, k=8,
+                                 n_shared=1, gate=SIGMOID, routed_scale=2.5, wdtype=E4M3),
+    "qwen2_skewed_prefill": Workload("qwen2_skewed_prefill", T=8192, H=2048, I=1408, E=60, k=4,
+                                     logits="zipf"),
+}
+
+
+def _rng(seed: int, name: str, index: int = 0) -> np.random.Generator:
+    return np.random.Generator(np.random.Philox(key=[seed, (zlib.crc32(name.encode()) << 20) + index]))
+
+
+def _normal(seed: int, name: str, index: int, shape, std: float) -> np.ndarray:
+    g = _rng(seed, name, index)
+    return g.standard_normal(size=shape, dtype=np.float32) * np.float32(std)
+
+
+def to_bf16_bits(a: np.ndarray) -> np.ndarray:
+    """Round fp32 to bf16 (nearest-even, torch's cast) and return the bits."""
+    return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(torch.bfloat16).view(
+        torch.int16).numpy().view(np.uint16)
+
+
+def bf16_bits_to_f32(b: np.ndarray) -> np.ndarray:
+    return (np.asarray(b, dtype=np.uint16).astype(np.uint32) << 16).view(np.float32)
+
+
+def to_e4m3_codes(a: np.ndarray) -> np.ndarray:
+    """fp32 values already inside [-448, 448] -> E4M3 codes (torch's cast)."""
+    t = torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).clamp_(-E4M3_MAX, E4M3_MAX)
+    return t.to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+
+
+def _threads() -> int:
+    return max(1, min(32, os.cpu_count() or 1))
+
+
+def _expert_matrix(seed, name, e, rows, cols, std, wdtype):
+    w = _normal(seed, name, e, (rows, cols), std)
+    if wdtype == BF16:
+        return to_bf16_bits(w), np.float32(1.0)
+    scale = np.float32(np.abs(w).max() / np.float32(E4M3_MAX))
+    return to_e4m3_codes(w / scale), scale
+
+
+def expert_weights(wl: Workload, which: str):
+    """Stacked expert weights: W13 [E_tot, 2I, H] (I gate rows then I up rows,
+    K-major) or W2 [E_tot, H, I]; plus per-expert fp32 scales (ones for bf16).
+    Shared experts follow the E routed ones."""
+    if which == "w13":
+        rows, cols, std = 2 * wl.I, wl.H, 1.0 / np.sqrt(wl.H)
+    else:
+        rows, cols, std = wl.H, wl.I, 1.0 / np.sqrt(wl.I)
+    dt = np.uint16 if wl.wdtype == BF16 else np.uint8
+    out = np.empty((wl.E_tot, rows, cols), dtype=dt)
+    scales = np.empty(wl.E_tot, dtype=np.float32)
+
+    def one(e):
+        m, s = _expert_matrix(wl.seed, which, e, rows, cols, std, wl.wdtype)
+        out[e] = m
+        scales[e] = s
+
+    with ThreadPoolExecutor(_threads()) as ex:
+        list(ex.map(one, range(wl.E_tot)))
+    return out, scales
+
+
+def tokens(wl: Workload) -> np.ndarray:
+    """x [T, H] bf16 bits, N(0,1)."""
+    return to_bf16_bits(_normal(wl.seed, "x", 0, (wl.T, wl.H), 1.0))
+
+
+def router_logits(wl: Workload, x_bits: np.ndarray) -> np.ndarray:
+    """Router logits [T, E] fp32 (an input of the layer)."""
+    if wl.logits == "zipf":
+        n = _normal(wl.seed, "logit_noise", 0, (wl.T, wl.E), 1.0).astype(np.float64)
+        r = np.arange(1, wl.E + 1, dtype=np.float64) ** (-wl.zipf_s)
+        bias = np.log(r / r.sum())
+        return (n + bias[None, :]).astype(np.float32)
+    wg = to_bf16_bits(_normal(wl.seed, "w_gate", 0, (wl.E, wl.H), 0.02))
+    xd = bf16_bits_to_f32(x_bits).astype(np.float64)
+    wd = bf16_bits_to_f32(wg).astype(np.float64)
+    return (xd @ wd.T).astype(np.float32)
+
+
+def activation_scale(x_bits: np.ndarray) -> float:
+    """Static per-tensor activation scale amax(x)/448 (fp32)."""
+    return float(np.float32(np.abs(bf16_bits_to_f32(x_bits)).max() / np.float32(E4M3_MAX)))
+
+
+def make_inputs(wl: Workload, weights: bool = True) -> dict:
+    """All inputs of one layer call (host numpy arrays)."""
+    x = tokens(wl)
+    d = {"x": x, "logits": router_logits(wl, x)}
+    if weights:
+        d["w13"], d["w13_scale"] = expert_weights(wl, "w13")
+        d["w2"], d["w2_scale"] = expert_weights(wl, "w2")
+    d["a1"] = activation_scale(x) if wl.adtype == E4M3 else 1.0
+    return d
+
+
+def random_rows(seed: int, name: str, rows: int, cols: int, dtype: int, std: float = 1.0):
+    """Stand-alone activation rows (bf16 bits or E4M3 codes) used to exercise a
+    single GEMM entry point in isolation."""
+    v = _normal(seed, name, 0, (rows, cols), std)
+    if dtype == BF16:
+        return to_bf16_bits(v)
+    return to_e4m3_codes(v / np.float32(np.abs(v).max() / E4M3_MAX))
+
+
+def random_f32(seed: int, name: str, shape, std: float = 1.0) -> np.ndarray:
+    return _normal(seed, name, 0, shape, std)
