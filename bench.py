@@ -1,0 +1,365 @@
+"""Throughput of the fused-MoE layer on B200.
+
+Default workload: the Mixtral-8x7B-shaped decode layer (T=64 tokens, H=4096,
+I=14336, E=8 experts, top-2 softmax, bf16 weights and activations), one
+moe_fused_forward per step with inputs resident in HBM.  Prints one JSON line.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                  [--workload NAME] [--T T]
+
+N > 1 (under torchrun): every rank runs an independent replica of the layer
+("replicas only": the single-GPU layer has no exchange step); value is the
+tokens of all ranks over the slowest rank's device time.
+--impl reference times the CPU oracle (the reference arm of this project) on
+a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from mixture_experts_layer_22_b200 import synthetic as syn  # noqa: E402
+
+METRIC = "fused-MoE layer tokens/s"
+UNIT = "tokens/s"
+
+
+def workload_desc(wl) -> str:
+    dt = {(0, 0): "bf16", (1, 1): "fp8 e4m3 w+a", (1, 0): "fp8 e4m3 w, bf16 a"}[(wl.wdtype, wl.adtype)]
+    gate = "softmax" if wl.gate == syn.SOFTMAX else f"sigmoid x{wl.routed_scale}"
+    sh = f" +{wl.n_shared} shared" if wl.n_shared else ""
+    return (f"{wl.name}: T={wl.T} H={wl.H} I={wl.I} E={wl.E} top-{wl.k} {gate}{sh}, {dt}")
+
+
+def config_of(wl, parallelism: str) -> dict:
+    return {"workload": workload_desc(wl), "T": wl.T, "H": wl.H, "I": wl.I, "E": wl.E, "k": wl.k,
+            "n_shared": wl.n_shared, "parallelism": parallelism,
+            "l2": "no flush: the step streams all active expert weights (GBs) through the 126 MB L2",
+            "inputs": "seeded synthetic (seed 0), resident in HBM before timing"}
+
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def weight_bytes_per_expert(wl) -> int:
+    esz = 2 if wl.wdtype == syn.BF16 else 1
+    return 3 * wl.H * wl.I * esz
+
+
+# ---------------------------------------------------------------- reference arm
+def cpu_oracle_rate(wl, d, budget_s: float = 15.0):
+    """Tokens/s of the oracle on this host, from a bounded token sample."""
+    import oracle as orc
+
+    def run(toks):
+        t0 = time.perf_counter()
+        orc.forward(d["x"], d["logits"], d["w13"], d["w2"], E=wl.E, k=wl.k, n_shared=wl.n_shared,
+                    gate=wl.gate, renorm=wl.renorm, routed_scale=wl.routed_scale, wdtype=wl.wdtype,
+                    adtype=wl.adtype, w13_scale=d["w13_scale"], w2_scale=d["w2_scale"],
+                    a1=float(d.get("a1", 1.0)), tokens=np.asarray(toks, np.int32))
+        return time.perf_counter() - t0
+
+    cores = orc.num_threads()
+    n = min(wl.T, cores)
+    dt = run(list(range(n)))
+    while dt < budget_s / 3 and n < wl.T:
+        n = min(wl.T, max(n + 1, int(n * min(4.0, budget_s / max(dt, 1e-3)))))
+        dt = run(list(range(n)))
+    return n / dt, cores, f"first {n} of {wl.T} tokens, {dt:.1f} s of host time"
+
+
+def reference_main(args, wl):
+    ws_n, rank, _ = dist_env()
+    if rank != 0:
+        return 0
+    d = syn.make_inputs(wl)
+    times = []
+    for _ in range(args.warmup):
+        cpu_oracle_rate(wl, d, budget_s=2.0)
+    rates = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        r, cores, sample = cpu_oracle_rate(wl, d, budget_s=args.ref_budget)
+        times.append(time.perf_counter() - t0)
+        rates.append(r)
+    value = statistics.median(rates)
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * wl.T / value,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": config_of(wl, "cpu oracle"),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.idx = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.QUERY}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def _read(self):
+        for ln in self.proc.stdout:
+            self.lines.append(ln.strip())
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.15)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- our arm
+def measured_peak_hbm():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return 6650.0, "fallback"
+
+
+def ours_main(args, wl):
+    import torch
+    import torch.distributed as dist
+
+    import mixture_experts_layer_22_b200 as moe
+
+    world, rank, local = dist_env()
+    if world > 1:
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", init_method="env://",
+                                timeout=__import__("datetime").timedelta(seconds=120))
+    dev = torch.device("cuda", local if world > 1 else 0)
+    torch.cuda.set_device(dev)
+    d = syn.make_inputs(wl)
+    shape = moe.Shape.of(wl)
+    esz = 2 if wl.wdtype == syn.BF16 else 1
+
+    def to_dev(a, u8=False):
+        t = torch.from_numpy(np.ascontiguousarray(a).view(np.int16 if not u8 else np.uint8)).to(dev)
+        return t if u8 else t.view(torch.bfloat16)
+
+    x = to_dev(d["x"])
+    logits = torch.from_numpy(d["logits"]).to(dev)
+    w13 = to_dev(d["w13"], u8=esz == 1)
+    w2 = to_dev(d["w2"], u8=esz == 1)
+    s13 = torch.from_numpy(d["w13_scale"]).to(dev) if esz == 1 else None
+    s2 = torch.from_numpy(d["w2_scale"]).to(dev) if esz == 1 else None
+    a1, a2 = float(d["a1"]), float(args.a2)
+    out = torch.empty((wl.T, wl.H), dtype=torch.bfloat16, device=dev)
+    ws = moe.workspace(shape, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        moe.fused_forward(shape, x, logits, w13, s13, w2, s2, a1, a2, out, ws, stream)
+
+    # routing facts for the roofline: distinct active experts and routed rows
+    E_t = wl.E + wl.n_shared
+    ids = torch.empty((wl.T, wl.k), dtype=torch.int32, device=dev)
+    wts = torch.empty((wl.T, wl.k), dtype=torch.float32, device=dev)
+    counts = torch.empty(E_t, dtype=torch.int32, device=dev)
+    offsets = torch.empty(E_t + 1, dtype=torch.int32, device=dev)
+    rows = torch.empty(moe.max_rows(shape), dtype=torch.int32, device=dev)
+    inv = torch.empty(wl.T * wl.k, dtype=torch.int32, device=dev)
+    moe.route_topk(shape, logits, ids, wts, stream)
+    moe.align_permute(shape, ids, counts, offsets, rows, inv, ws, stream)
+    torch.cuda.synchronize(dev)
+    active = int((counts.cpu() > 0).sum())
+    slots = int(offsets[-1].item())
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    launches_per_step = moe.last_launch_count()
+    st = moe.device_status(ws, stream)
+    if st != 0:
+        raise SystemExit(f"device status after warm-up: {moe.status_string(st)}")
+
+    clocks = ClockSampler(dev.index if world == 1 else local)
+    clocks.start()
+    time.sleep(0.3)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for _ in range(args.steps):
+        step()
+    ev1.record(stream)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop()
+    ms = ev0.elapsed_time(ev1)
+    if world > 1:
+        t = torch.tensor([ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    ms_per_step = ms / args.steps
+    value = world * wl.T * args.steps / (ms / 1e3)
+
+    # per-kernel device time of the two expert GEMMs (same inputs, step-wise calls)
+    xp = torch.empty((moe.max_rows(shape), wl.H * (1 if wl.adtype else 2)), dtype=torch.uint8, device=dev)
+    hb = torch.empty((moe.max_rows(shape), wl.I * (1 if wl.adtype else 2)), dtype=torch.uint8, device=dev)
+    yb = torch.empty((moe.max_rows(shape), wl.H), dtype=torch.float32, device=dev)
+    moe.gather(shape, x, rows, offsets, a1, xp, stream)
+    g1 = [torch.cuda.Event(enable_timing=True) for _ in range(2 * args.steps)]
+    g2 = [torch.cuda.Event(enable_timing=True) for _ in range(2 * args.steps)]
+    for i in range(args.steps + 1):
+        j = i - 1
+        if j >= 0:
+            g1[2 * j].record(stream)
+        moe.grouped_gemm_swiglu(shape, xp, w13, s13, a1, a2, offsets, hb, ws, stream)
+        if j >= 0:
+            g1[2 * j + 1].record(stream)
+            g2[2 * j].record(stream)
+        moe.grouped_gemm_down(shape, hb, w2, s2, a2, offsets, yb, ws, stream)
+        if j >= 0:
+            g2[2 * j + 1].record(stream)
+    torch.cuda.synchronize(dev)
+    t_g1 = statistics.mean(g1[2 * j].elapsed_time(g1[2 * j + 1]) for j in range(args.steps))
+    t_g2 = statistics.mean(g2[2 * j].elapsed_time(g2[2 * j + 1]) for j in range(args.steps))
+    w13_bytes = active * 2 * wl.H * wl.I * esz
+    w2_bytes = active * wl.H * wl.I * esz
+    aesz = 1 if wl.adtype else 2
+    g1_bytes = w13_bytes + slots * wl.H * aesz + slots * wl.I * aesz
+    g2_bytes = w2_bytes + slots * wl.I * aesz + slots * wl.H * 4
+    peak, peak_kind = measured_peak_hbm()
+    ach = g1_bytes / (t_g1 * 1e-3) / 1e9
+    layer_bytes = active * weight_bytes_per_expert(wl) + wl.T * wl.H * 2 * 2 + wl.T * wl.E * 4
+    flops = 2.0 * 3 * wl.H * wl.I * (wl.T * wl.k + wl.n_shared * wl.T)
+
+    # end to end through the C ABI with host buffers: pinned H2D of x and
+    # logits, the fused call, D2H of out, every step
+    hx = torch.from_numpy(d["x"].view(np.int16)).view(torch.bfloat16).pin_memory()
+    hl = torch.from_numpy(d["logits"]).pin_memory()
+    ho = torch.empty((wl.T, wl.H), dtype=torch.bfloat16).pin_memory()
+    dx = torch.empty_like(x)
+    dl = torch.empty_like(logits)
+
+    def e2e_step():
+        dx.copy_(hx, non_blocking=True)
+        dl.copy_(hl, non_blocking=True)
+        moe.fused_forward(shape, dx, dl, w13, s13, w2, s2, a1, a2, out, ws, stream)
+        ho.copy_(out, non_blocking=True)
+
+    for _ in range(args.warmup):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+        stream.synchronize()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    ems = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([ems], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ems = float(t.item())
+    e2e_val = world * wl.T * args.steps / (ems / 1e3)
+
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": {(0, 0): "bf16", (1, 1): "e4m3", (1, 0): "e4m3w-bf16a"}[(wl.wdtype, wl.adtype)],
+        "data": "synthetic", "config": config_of(wl, f"replicas x{world}" if world > 1 else "1 GPU"),
+        "hbm_gbs": layer_bytes / (ms_per_step * 1e-3) / 1e9, "tflops": flops / (ms_per_step * 1e-3) / 1e12,
+        "active_experts": active,
+        "roofline": {"bound": "hbm", "kernel": "grouped_gemm (gate/up + SwiGLU)", "achieved": ach,
+                     "peak": peak, "peak_kind": peak_kind, "unit": "GB/s", "frac": ach / peak,
+                     "traffic": None, "algorithmic_bytes": g1_bytes, "ms": t_g1,
+                     "down_ms": t_g2, "down_gbs": g2_bytes / (t_g2 * 1e-3) / 1e9},
+        "e2e": {"value": e2e_val, "unit": UNIT, "h2d_bytes_per_step": int(hx.numel() * 2 + hl.numel() * 4),
+                "d2h_bytes_per_step": int(ho.numel() * 2)},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clk,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu:
+        r, cores, sample = cpu_oracle_rate(wl, d, budget_s=args.ref_budget)
+        line["cpu_baseline"] = {"value": r, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample}
+    if world > 1:
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="mixtral_decode", choices=sorted(syn.WORKLOADS))
+    ap.add_argument("--T", type=int, default=None)
+    ap.add_argument("--a2", type=float, default=1.0, help="static hidden-activation scale (FP8 activations)")
+    ap.add_argument("--ref-budget", type=float, default=15.0, help="seconds of host time per oracle sample")
+    ap.add_argument("--no-cpu", action="store_true", help="skip the cpu_baseline leg")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    wl = syn.WORKLOADS[args.workload]
+    if args.T is not None:
+        wl = wl.with_T(args.T)
+    if args.impl == "reference":
+        return reference_main(args, wl)
+    return ours_main(args, wl)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

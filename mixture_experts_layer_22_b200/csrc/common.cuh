@@ -1,0 +1,78 @@
+// common.cuh - internal declarations shared by the library's translation units.
+#pragma once
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "moe.h"
+
+namespace moe {
+
+constexpr int kMaxExperts = 512;            // routed experts per layer
+constexpr int kMaxExpertsTotal = kMaxExperts + 1;
+constexpr int kMaxTopK = 32;
+constexpr int kMaxCtas = 160;               // persistent GEMM grid bound (>= SM count)
+constexpr int kAlignChunk = 1024;           // routed rows per align block
+
+// Control words at the start of the workspace.
+struct Ctrl {
+    int32_t status;       // first device-side error (moe_status), 0 = none
+    int32_t ticket;       // align: blocks finished counting
+    int32_t pad_[62];
+};
+
+__device__ __forceinline__ void set_status(int32_t *status, int32_t code)
+{
+    atomicCAS(status, 0, code);
+}
+
+// Workspace carving (host side), every region 256-byte aligned.
+struct WsLayout {
+    size_t ctrl, ids, w, counts, offsets, chunk_hist, chunk_base, sorted_rows, inv;
+    size_t xp, h, y, counters, partials;
+    size_t total;
+    int64_t max_rows;
+    int n_chunks;
+    int acc_cols;         // accumulator columns of the widest GEMM tile
+};
+
+// Which GEMM kernel a call uses.
+struct GemmPlan {
+    bool swap;            // weights in the MMA M slot, tokens in N
+    int bn;               // Swap-AB: token rows per tile (16..256); normal: 256
+};
+
+GemmPlan plan_gemm(const moe_shape_t &s);
+bool ws_layout(const moe_shape_t &s, WsLayout &L);
+int validate_shape(const moe_shape_t *s, bool need_gemm);
+
+// ---- launchers (return cudaError_t of the launch) ----
+cudaError_t launch_route(const moe_shape_t &s, const float *logits, int32_t *ids, float *w,
+                         cudaStream_t st);
+cudaError_t launch_align(const moe_shape_t &s, const int32_t *ids, int32_t *counts,
+                         int32_t *offsets, int32_t *sorted_rows, int32_t *inv, int32_t *chunk_hist,
+                         int32_t *chunk_base, Ctrl *ctrl, cudaStream_t st, int *launches);
+cudaError_t launch_gather(const moe_shape_t &s, const void *x, const int32_t *sorted_rows,
+                          const int32_t *offsets, float a1, void *xp, int64_t max_rows,
+                          cudaStream_t st);
+cudaError_t launch_combine(const moe_shape_t &s, const float *y, const float *w,
+                           const int32_t *inv, const int32_t *offsets, void *out,
+                           cudaStream_t st);
+
+struct GemmArgs {
+    int mode;                 // 0: gate/up + SwiGLU, 1: down projection
+    const void *act;          // xp or h
+    const void *wgt;          // w13 or w2
+    const float *wscale;
+    float ascale, qscale;
+    const int32_t *offsets;
+    void *out;
+    int32_t *status;
+    int32_t *counters;
+    float *partials;
+    int64_t max_rows;
+};
+cudaError_t launch_grouped_gemm(const moe_shape_t &s, const GemmPlan &p, const GemmArgs &a,
+                                cudaStream_t st, int *launches, int *host_err);
+
+}  // namespace moe

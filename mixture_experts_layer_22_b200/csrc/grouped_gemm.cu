@@ -1,0 +1,741 @@
+// grouped_gemm.cu - persistent grouped expert GEMM on the 5th-generation
+// tensor cores (tcgen05 + tensor memory), fed by TMA.
+//
+// What it computes (the two expert GEMMs of the fused-MoE layer):
+//   mode 0:  h_s = SiLU(sc * xp_s . W1[e]^T) * (sc * xp_s . W3[e]^T)
+//   mode 1:  y_s = sc * h_s . W2[e]^T
+// for every row s of expert e's segment of the permuted activations, with fp32
+// accumulation and sc = activation scale * per-expert weight scale.
+//
+// Operand order ("Swap-AB", from "Mixture-of-Experts kernel engineering on
+// Amazon SageMaker AI", abstract, the B^T[N,K] x A^T[K,M] = C^T[N,M] passage,
+// and the Russian summary's section "Swap-AB: развернуть матрицы под WGMMA"):
+// the tensor core's M extent is fixed (128 rows for a one-CTA tcgen05.mma),
+// so when an expert sees few token rows the kernel puts 128 expert-weight rows
+// in M and the token rows in N (16..256, chosen per tile at run time).  The
+// normal order puts 128 token rows in M and 256 weight rows in N.  Both give
+// the same result up to fp32 summation order.
+//
+// Structure (one CTA per SM, 192 threads):
+//   warp 0      TMA producer: weight and activation tiles into a smem ring
+//   warp 1      tcgen05.mma issuer (one thread) and tensor-memory owner
+//   warps 2..5  epilogue: tcgen05.ld the fp32 accumulator, scale, SwiGLU,
+//               convert and store
+// Accumulators are double-buffered in tensor memory so the epilogue of one
+// tile overlaps the main loop of the next.  Work is split over the grid as
+// whole tiles for all full rounds and, for the remaining tiles, as equal
+// contiguous ranges of K-steps ("stream-K"); a tile split across CTAs is
+// finished by the last CTA to arrive, which sums the fp32 partials in a fixed
+// CTA order (deterministic).  The tile list is derived on the device from the
+// segment offsets, so token counts are run-time values and nothing is
+// recompiled per batch size.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_fp8.h>
+
+#include <mutex>
+
+#include "common.cuh"
+#include "ptx.cuh"
+
+namespace moe {
+
+struct GemmParams {
+    const int32_t *offsets;
+    int E_tot;
+    int K;            // reduction length in elements
+    int n_feat;       // mode 0: I (hidden features); mode 1: H (outputs)
+    int w_rows;       // weight rows per expert: 2I (mode 0) or H (mode 1)
+    int out_ld;       // row stride of the output, elements
+    void *out;
+    const float *wscale;
+    float ascale;     // activation scale (1 for bf16 activations)
+    float qscale;     // mode 0 with E4M3 output: h is stored as e4m3(h / qscale)
+    int32_t *status;
+    int32_t *counters;
+    float *partials;
+    int stream_k;     // 0: whole tiles only
+};
+
+template <int kMode, bool kSwap, bool kFp8, int kBN>
+struct Cfg {
+    static constexpr int kStageA = 128 * 128;               // 128 rows x 128 bytes
+    static constexpr int kStageB = kBN * 128;
+    static constexpr int kStage = kStageA + kStageB;
+    static constexpr int kDynBudget = 205 * 1024;
+    static constexpr int kStagesRaw = kDynBudget / kStage;
+    static constexpr int kStages = kStagesRaw > 12 ? 12 : kStagesRaw;
+    static constexpr int kDynSmem = kStages * kStage + 1024;
+    static constexpr int kAccCols = kSwap ? kBN : 256;      // fp32 columns per accumulator
+    static constexpr int kTmemCols = (2 * kAccCols) <= 32 ? 32 : 2 * kAccCols;
+    static constexpr int kRowsTile = kSwap ? kBN : 128;     // token rows per tile
+    static constexpr int kFeatTile = kMode == 0 ? (kSwap ? 64 : 128) : (kSwap ? 128 : 256);
+    static constexpr int kKStage = kFp8 ? 128 : 64;         // elements per 128-byte row
+    static constexpr uint32_t kFmt = kFp8 ? 0u : 1u;
+    static_assert(kStages >= 2, "smem ring too small");
+    static_assert(kTmemCols <= 512, "tensor memory");
+};
+
+// Work item: one tile (expert e, feature tile ft, row tile rt) over K-steps
+// [kb, ke).  `partial` is set when the item is one CTA's share of a split tile.
+struct Item {
+    int e, ft, rt, kb, ke;
+    int partial;
+    int sk_tile;       // index among stream-K tiles (counters / fixup)
+    int slot;          // this CTA's partial slot
+};
+
+struct Sched {
+    int n_tiles, KT, G, dp_tiles, sk_tiles, sk_ctas;
+    long long sk_total;
+};
+
+// Smallest CTA index whose stream-K range contains K-step `i`.
+__device__ __forceinline__ int sk_cta_of(long long i, const Sched &S)
+{
+    return static_cast<int>(((i + 1) * S.sk_ctas + S.sk_total - 1) / S.sk_total) - 1;
+}
+
+__device__ __forceinline__ long long sk_begin(int c, const Sched &S)
+{
+    return static_cast<long long>(c) * S.sk_total / S.sk_ctas;
+}
+
+// Iterator over the work items of CTA `c`: whole tiles c, c+G, ... below
+// dp_tiles, then its contiguous K-step range of the stream-K region.
+struct ItemIter {
+    int c, i_dp;
+    long long it, it_end;
+    bool in_sk, first_sk;
+};
+
+__device__ __forceinline__ void iter_init(ItemIter &I, const Sched &S, int c)
+{
+    I.c = c;
+    I.i_dp = 0;
+    I.in_sk = false;
+    I.first_sk = true;
+    if (c < S.sk_ctas) {
+        I.it = sk_begin(c, S);
+        I.it_end = sk_begin(c + 1, S);
+    } else {
+        I.it = I.it_end = 0;
+    }
+}
+
+template <int kRowsTile, int kFeatTileUnused>
+__device__ __forceinline__ void tile_coords(int t, const int *s_prefix, const int *s_off, int Et,
+                                            int n_ft, int &e, int &ft, int &rt)
+{
+    int lo = 0, hi = Et - 1;                 // largest e with prefix[e] <= t
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (s_prefix[mid] <= t) lo = mid;
+        else hi = mid - 1;
+    }
+    e = lo;
+    const int seg = s_off[e + 1] - s_off[e];
+    const int nrt = (seg + kRowsTile - 1) / kRowsTile;
+    const int local = t - s_prefix[e];
+    rt = local % nrt;
+    ft = local / nrt;
+}
+
+template <int kRowsTile>
+__device__ __forceinline__ bool iter_next(ItemIter &I, const Sched &S, const int *s_prefix,
+                                          const int *s_off, int Et, int n_ft, Item &out)
+{
+    if (!I.in_sk) {
+        const int t = I.c + I.i_dp * S.G;
+        if (t < S.dp_tiles) {
+            ++I.i_dp;
+            tile_coords<kRowsTile, 0>(t, s_prefix, s_off, Et, n_ft, out.e, out.ft, out.rt);
+            out.kb = 0;
+            out.ke = S.KT;
+            out.partial = 0;
+            out.sk_tile = -1;
+            out.slot = -1;
+            return true;
+        }
+        I.in_sk = true;
+    }
+    if (I.it >= I.it_end) return false;
+    const int tl = static_cast<int>(I.it / S.KT);
+    const int kb = static_cast<int>(I.it % S.KT);
+    const long long left = I.it_end - I.it;
+    const int ke = static_cast<int>(left < S.KT - kb ? kb + left : S.KT);
+    tile_coords<kRowsTile, 0>(S.dp_tiles + tl, s_prefix, s_off, Et, n_ft, out.e, out.ft, out.rt);
+    out.kb = kb;
+    out.ke = ke;
+    out.partial = !(kb == 0 && ke == S.KT);
+    out.sk_tile = tl;
+    out.slot = 2 * I.c + (I.first_sk ? 0 : 1);
+    I.first_sk = false;
+    I.it += ke - kb;
+    return true;
+}
+
+__device__ __forceinline__ float silu_mul(float g, float u)
+{
+    return g / (1.0f + __expf(-g)) * u;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float a, float b)
+{
+    const __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
+    return *reinterpret_cast<const uint32_t *>(&v);
+}
+
+__device__ __forceinline__ uint32_t e4m3_code(float v)
+{
+    return static_cast<uint32_t>(__nv_cvt_float_to_fp8(v, __NV_SATFINITE, __NV_E4M3)) & 0xFFu;
+}
+
+template <int kMode, bool kSwap, bool kFp8, int kBN>
+__global__ void __launch_bounds__(192, 1)
+    grouped_gemm_kernel(const __grid_constant__ CUtensorMap tm_w,
+                        const __grid_constant__ CUtensorMap tm_x, GemmParams p)
+{
+    using C = Cfg<kMode, kSwap, kFp8, kBN>;
+    extern __shared__ uint8_t dyn_smem[];
+    __shared__ int s_off[kMaxExpertsTotal + 1];
+    __shared__ int s_prefix[kMaxExpertsTotal + 1];
+    __shared__ __align__(8) uint64_t s_full[C::kStages], s_empty[C::kStages];
+    __shared__ __align__(8) uint64_t s_tfull[2], s_tempty[2], s_drain;
+    __shared__ uint32_t s_tmem_base;
+    __shared__ volatile int s_abort;
+    __shared__ int s_is_last;
+    __shared__ float s_xchg[kMode == 0 && kSwap ? 16 * 64 : 1];
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int Et = p.E_tot;
+    uint8_t *tiles = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(dyn_smem) + 1023) &
+                                                 ~static_cast<uintptr_t>(1023));
+
+    // ---- set-up: barriers, tensor memory, tile table ----
+    if (threadIdx.x == 0) {
+        s_abort = 0;
+        for (int i = 0; i < C::kStages; ++i) {
+            mbar_init(smem_u32(&s_full[i]), 1);
+            mbar_init(smem_u32(&s_empty[i]), 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(smem_u32(&s_tfull[i]), 1);
+            mbar_init(smem_u32(&s_tempty[i]), 4);
+        }
+        mbar_init(smem_u32(&s_drain), 1);
+        fence_mbar_init();
+        prefetch_tmap(&tm_w);
+        prefetch_tmap(&tm_x);
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_u32(&s_tmem_base), C::kTmemCols);
+        tmem_relinquish();
+    }
+    const int n_ft = (p.n_feat + C::kFeatTile - 1) / C::kFeatTile;
+    if (warp == 2) {
+        for (int e = lane; e <= Et; e += 32) s_off[e] = p.offsets[e];
+        __syncwarp();
+        const int per = (Et + 31) / 32;
+        const int lo = min(Et, lane * per), hi = min(Et, lo + per);
+        int sum = 0;
+        bool bad = false;
+        for (int e = lo; e < hi; ++e) {
+            const int seg = s_off[e + 1] - s_off[e];
+            if (seg < 0 || (seg & 15) != 0 || (s_off[e] & 15) != 0) bad = true;
+            sum += seg > 0 ? ((seg + C::kRowsTile - 1) / C::kRowsTile) * n_ft : 0;
+        }
+        int inc = sum;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(0xffffffffu, inc, o);
+            if (lane >= o) inc += v;
+        }
+        int run = inc - sum;
+        for (int e = lo; e < hi; ++e) {
+            s_prefix[e] = run;
+            const int seg = s_off[e + 1] - s_off[e];
+            run += seg > 0 ? ((seg + C::kRowsTile - 1) / C::kRowsTile) * n_ft : 0;
+        }
+        if (lane == 31) s_prefix[Et] = inc;
+        if (__any_sync(0xffffffffu, bad) && lane == 0) {
+            set_status(p.status, MOE_ERR_DEVICE_CHECK);
+            s_prefix[Et] = 0;   // no work: refuse mis-aligned segments
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = s_tmem_base;
+
+    Sched S;
+    S.n_tiles = s_prefix[Et];
+    S.KT = p.K / C::kKStage;
+    S.G = gridDim.x;
+    if (!p.stream_k || S.n_tiles % S.G == 0) S.dp_tiles = S.n_tiles;
+    else if (S.n_tiles <= S.G) S.dp_tiles = 0;
+    else S.dp_tiles = (S.n_tiles / S.G - 1) * S.G;
+    S.sk_tiles = S.n_tiles - S.dp_tiles;
+    S.sk_total = static_cast<long long>(S.sk_tiles) * S.KT;
+    S.sk_ctas = static_cast<int>(S.sk_total < S.G ? S.sk_total : S.G);
+
+    if (warp == 0) {
+        // ================= TMA producer =================
+        if (lane == 0) {
+            const uint64_t pol_w = policy_evict_first();
+            const uint64_t pol_x = policy_evict_last();
+            int stage = 0;
+            uint32_t phase = 0;
+            int in_flight = 0;
+            ItemIter I;
+            iter_init(I, S, blockIdx.x);
+            Item it;
+            bool ok = true;
+            while (ok && iter_next<C::kRowsTile>(I, S, s_prefix, s_off, Et, n_ft, it)) {
+                const int row0 = s_off[it.e] + it.rt * C::kRowsTile;
+                const int wbase = it.e * p.w_rows;
+                for (int kk = it.kb; kk < it.ke; ++kk) {
+                    if (!mbar_wait(smem_u32(&s_empty[stage]), phase ^ 1u, &s_abort)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t fb = smem_u32(&s_full[stage]);
+                    mbar_arrive_expect_tx(fb, C::kStage);
+                    const uint32_t sa = smem_u32(tiles + stage * C::kStage);
+                    const uint32_t sb = sa + C::kStageA;
+                    const int kx = kk * C::kKStage;
+                    if (kSwap) {
+                        if (kMode == 0) {
+                            tma_load_2d(sa, &tm_w, fb, kx, wbase + it.ft * 64, pol_w);
+                            tma_load_2d(sa + 64 * 128, &tm_w, fb, kx, wbase + p.n_feat + it.ft * 64, pol_w);
+                        } else {
+                            tma_load_2d(sa, &tm_w, fb, kx, wbase + it.ft * 128, pol_w);
+                        }
+                        tma_load_2d(sb, &tm_x, fb, kx, row0, pol_x);
+                    } else {
+                        tma_load_2d(sa, &tm_x, fb, kx, row0, pol_x);
+                        if (kMode == 0) {
+                            tma_load_2d(sb, &tm_w, fb, kx, wbase + it.ft * 128, pol_w);
+                            tma_load_2d(sb + 128 * 128, &tm_w, fb, kx, wbase + p.n_feat + it.ft * 128, pol_w);
+                        } else {
+                            tma_load_2d(sb, &tm_w, fb, kx, wbase + it.ft * 256, pol_w);
+                        }
+                    }
+                    ++in_flight;
+                    if (++stage == C::kStages) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+            if (!ok) {
+                // let copies already issued land before the CTA can exit
+                int st = stage;
+                uint32_t ph = phase;
+                for (int i = 0; i < C::kStages && i < in_flight; ++i) {
+                    st = st == 0 ? C::kStages - 1 : st - 1;
+                    if (st == C::kStages - 1) ph ^= 1u;
+                    volatile int no_abort = 0;
+                    mbar_wait(smem_u32(&s_full[st]), ph, &no_abort);
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ================= MMA issuer =================
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            int acc = 0;
+            uint32_t acc_phase = 0;
+            ItemIter I;
+            iter_init(I, S, blockIdx.x);
+            Item it;
+            bool ok = true;
+            while (ok && iter_next<C::kRowsTile>(I, S, s_prefix, s_off, Et, n_ft, it)) {
+                if (!mbar_wait(smem_u32(&s_tempty[acc]), acc_phase ^ 1u, &s_abort)) break;
+                tc_fence_after();
+                const uint32_t d = tmem_base + acc * C::kAccCols;
+                int n = 256;
+                if (kSwap) {
+                    const int seg = s_off[it.e + 1] - s_off[it.e];
+                    n = min(C::kRowsTile, seg - it.rt * C::kRowsTile);
+                }
+                const uint32_t idesc = idesc_make(C::kFmt, 128, n);
+                for (int kk = it.kb; kk < it.ke; ++kk) {
+                    if (!mbar_wait(smem_u32(&s_full[stage]), phase, &s_abort)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t sa = smem_u32(tiles + stage * C::kStage);
+                    const uint32_t sb = sa + C::kStageA;
+#pragma unroll
+                    for (int s = 0; s < 4; ++s) {
+                        const uint64_t ad = sdesc_k_sw128(sa + s * 32);
+                        const uint64_t bd = sdesc_k_sw128(sb + s * 32);
+                        const uint32_t accum = (kk > it.kb || s > 0) ? 1u : 0u;
+                        if (kFp8) mma_e4m3(d, ad, bd, idesc, accum);
+                        else mma_bf16(d, ad, bd, idesc, accum);
+                    }
+                    mma_commit(smem_u32(&s_empty[stage]));
+                    if (++stage == C::kStages) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                if (!ok) break;
+                mma_commit(smem_u32(&s_tfull[acc]));
+                if (++acc == 2) {
+                    acc = 0;
+                    acc_phase ^= 1u;
+                }
+            }
+            // every MMA issued above has completed once this barrier fires
+            mma_commit(smem_u32(&s_drain));
+            volatile int no_abort = 0;
+            mbar_wait(smem_u32(&s_drain), 0, &no_abort);
+        }
+    } else {
+        // ================= epilogue (warps 2..5) =================
+        const int q = warp & 3;                 // tensor-memory lane quarter
+        const int r = q * 32 + lane;            // accumulator row of this thread
+        const int etid = threadIdx.x - 64;      // 0..127
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        ItemIter I;
+        iter_init(I, S, blockIdx.x);
+        Item it;
+        while (iter_next<C::kRowsTile>(I, S, s_prefix, s_off, Et, n_ft, it)) {
+            const bool got = mbar_wait(smem_u32(&s_tfull[acc]), acc_phase, &s_abort);
+            if (!named_bar_and(1, 128, got)) break;   // all four warps agree
+            tc_fence_after();
+            const int seg = s_off[it.e + 1] - s_off[it.e];
+            const int row0 = s_off[it.e] + it.rt * C::kRowsTile;
+            const int rows = min(C::kRowsTile, seg - it.rt * C::kRowsTile);
+            const float sc = p.ascale * (p.wscale ? __ldg(&p.wscale[it.e]) : 1.0f);
+            const uint32_t tacc = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * C::kAccCols;
+            const int ncols = kSwap ? rows : 256;
+            if (!it.partial) {
+                if (kSwap && kMode == 0) {
+                    // rows 0..63 gate, 64..127 up for features f0 .. f0+63
+                    const int f0 = it.ft * 64;
+                    for (int c0 = 0; c0 < ncols; c0 += 16) {
+                        uint32_t v[16];
+                        tmem_ld16(tacc + c0, v);
+                        tmem_wait_ld();
+                        if (q >= 2)
+#pragma unroll
+                            for (int j = 0; j < 16; ++j) s_xchg[j * 64 + (r - 64)] = __uint_as_float(v[j]);
+                        named_bar_sync(1, 128);
+                        if (q < 2) {
+#pragma unroll
+                            for (int j = 0; j < 16; ++j) {
+                                const float g = __uint_as_float(v[j]) * sc;
+                                const float u = s_xchg[j * 64 + r] * sc;
+                                const float hv = silu_mul(g, u);
+                                const size_t o = static_cast<size_t>(row0 + c0 + j) * p.out_ld + f0 + r;
+                                if (kFp8)
+                                    static_cast<uint8_t *>(p.out)[o] = static_cast<uint8_t>(e4m3_code(hv / p.qscale));
+                                else
+                                    static_cast<__nv_bfloat16 *>(p.out)[o] = __float2bfloat16_rn(hv);
+                            }
+                        }
+                        named_bar_sync(1, 128);
+                    }
+                } else if (kSwap) {
+                    const int h0 = it.ft * 128;
+                    for (int c0 = 0; c0 < ncols; c0 += 16) {
+                        uint32_t v[16];
+                        tmem_ld16(tacc + c0, v);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int j = 0; j < 16; ++j)
+                            static_cast<float *>(p.out)[static_cast<size_t>(row0 + c0 + j) * p.out_ld + h0 + r] =
+                                __uint_as_float(v[j]) * sc;
+                    }
+                } else if (kMode == 0) {
+                    const int f0 = it.ft * 128;
+                    const bool valid = r < rows;
+                    for (int c0 = 0; c0 < 128; c0 += 16) {
+                        uint32_t g[16], u[16];
+                        tmem_ld16(tacc + c0, g);
+                        tmem_ld16(tacc + 128 + c0, u);
+                        tmem_wait_ld();
+                        if (valid) {
+                            float hv[16];
+#pragma unroll
+                            for (int j = 0; j < 16; ++j)
+                                hv[j] = silu_mul(__uint_as_float(g[j]) * sc, __uint_as_float(u[j]) * sc);
+                            const size_t o = static_cast<size_t>(row0 + r) * p.out_ld + f0 + c0;
+                            if (kFp8) {
+                                uint32_t w4[4];
+#pragma unroll
+                                for (int j = 0; j < 4; ++j)
+                                    w4[j] = e4m3_code(hv[4 * j] / p.qscale) | (e4m3_code(hv[4 * j + 1] / p.qscale) << 8) |
+                                            (e4m3_code(hv[4 * j + 2] / p.qscale) << 16) |
+                                            (e4m3_code(hv[4 * j + 3] / p.qscale) << 24);
+                                *reinterpret_cast<uint4 *>(static_cast<uint8_t *>(p.out) + o) =
+                                    make_uint4(w4[0], w4[1], w4[2], w4[3]);
+                            } else {
+                                uint32_t w8[8];
+#pragma unroll
+                                for (int j = 0; j < 8; ++j) w8[j] = pack_bf16x2(hv[2 * j], hv[2 * j + 1]);
+                                uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(p.out) + o);
+                                dst[0] = make_uint4(w8[0], w8[1], w8[2], w8[3]);
+                                dst[1] = make_uint4(w8[4], w8[5], w8[6], w8[7]);
+                            }
+                        }
+                    }
+                } else {
+                    const int h0 = it.ft * 256;
+                    const bool valid = r < rows;
+                    for (int c0 = 0; c0 < 256; c0 += 16) {
+                        if (h0 + c0 >= p.n_feat) break;
+                        uint32_t v[16];
+                        tmem_ld16(tacc + c0, v);
+                        tmem_wait_ld();
+                        if (valid) {
+                            float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(p.out) +
+                                                                     static_cast<size_t>(row0 + r) * p.out_ld + h0 + c0);
+#pragma unroll
+                            for (int j = 0; j < 4; ++j)
+                                dst[j] = make_float4(__uint_as_float(v[4 * j]) * sc, __uint_as_float(v[4 * j + 1]) * sc,
+                                                     __uint_as_float(v[4 * j + 2]) * sc, __uint_as_float(v[4 * j + 3]) * sc);
+                        }
+                    }
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_u32(&s_tempty[acc]));
+            } else {
+                // ---- one share of a split tile: store the raw partial ----
+                float *slot = p.partials + static_cast<size_t>(it.slot) * 128 * C::kAccCols;
+                for (int c0 = 0; c0 < ncols; c0 += 16) {
+                    uint32_t v[16];
+                    tmem_ld16(tacc + c0, v);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) __stcg(&slot[(c0 + j) * 128 + r], __uint_as_float(v[j]));
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_u32(&s_tempty[acc]));
+                __threadfence();
+                named_bar_sync(1, 128);
+                // contributing CTAs of this tile, in K order
+                const long long t_it0 = static_cast<long long>(it.sk_tile) * S.KT;
+                const int c_first = sk_cta_of(t_it0, S);
+                const int c_last = sk_cta_of(t_it0 + S.KT - 1, S);
+                if (etid == 0) {
+                    const int old = atomicAdd(&p.counters[it.sk_tile], 1);
+                    s_is_last = (old == c_last - c_first);
+                }
+                named_bar_sync(1, 128);
+                if (s_is_last) {
+                    __threadfence();
+                    auto slot_of = [&](int c) -> const float * {
+                        const int first_tile = static_cast<int>(sk_begin(c, S) / S.KT);
+                        const int sidx = 2 * c + (first_tile == it.sk_tile ? 0 : 1);
+                        return p.partials + static_cast<size_t>(sidx) * 128 * C::kAccCols;
+                    };
+                    if (kSwap && kMode == 0) {
+                        const int f0 = it.ft * 64;
+                        const int rr = etid & 63;
+                        for (int j = etid >> 6; j < ncols; j += 2) {
+                            float g = 0.f, u = 0.f;
+                            for (int c = c_first; c <= c_last; ++c) {
+                                const float *ps = slot_of(c);
+                                g += __ldcg(&ps[j * 128 + rr]);
+                                u += __ldcg(&ps[j * 128 + 64 + rr]);
+                            }
+                            const float hv = silu_mul(g * sc, u * sc);
+                            const size_t o = static_cast<size_t>(row0 + j) * p.out_ld + f0 + rr;
+                            if (kFp8) static_cast<uint8_t *>(p.out)[o] = static_cast<uint8_t>(e4m3_code(hv / p.qscale));
+                            else static_cast<__nv_bfloat16 *>(p.out)[o] = __float2bfloat16_rn(hv);
+                        }
+                    } else if (kSwap) {
+                        const int h0 = it.ft * 128;
+                        for (int j = 0; j < ncols; ++j) {
+                            float a = 0.f;
+                            for (int c = c_first; c <= c_last; ++c) a += __ldcg(&slot_of(c)[j * 128 + etid]);
+                            static_cast<float *>(p.out)[static_cast<size_t>(row0 + j) * p.out_ld + h0 + etid] = a * sc;
+                        }
+                    } else if (kMode == 0) {
+                        const int f0 = it.ft * 128;
+                        if (etid < rows)
+                            for (int j = 0; j < 128; ++j) {
+                                float g = 0.f, u = 0.f;
+                                for (int c = c_first; c <= c_last; ++c) {
+                                    const float *ps = slot_of(c);
+                                    g += __ldcg(&ps[j * 128 + etid]);
+                                    u += __ldcg(&ps[(128 + j) * 128 + etid]);
+                                }
+                                const float hv = silu_mul(g * sc, u * sc);
+                                const size_t o = static_cast<size_t>(row0 + etid) * p.out_ld + f0 + j;
+                                if (kFp8) static_cast<uint8_t *>(p.out)[o] = static_cast<uint8_t>(e4m3_code(hv / p.qscale));
+                                else static_cast<__nv_bfloat16 *>(p.out)[o] = __float2bfloat16_rn(hv);
+                            }
+                    } else {
+                        const int h0 = it.ft * 256;
+                        if (etid < rows)
+                            for (int j = 0; j < 256 && h0 + j < p.n_feat; ++j) {
+                                float a = 0.f;
+                                for (int c = c_first; c <= c_last; ++c) a += __ldcg(&slot_of(c)[j * 128 + etid]);
+                                static_cast<float *>(p.out)[static_cast<size_t>(row0 + etid) * p.out_ld + h0 + j] = a * sc;
+                            }
+                    }
+                }
+                named_bar_sync(1, 128);
+            }
+            if (++acc == 2) {
+                acc = 0;
+                acc_phase ^= 1u;
+            }
+        }
+    }
+
+    // ---- tear-down ----
+    tc_fence_before();
+    __syncthreads();
+    if (threadIdx.x == 0 && s_abort) set_status(p.status, MOE_ERR_TIMEOUT);
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, C::kTmemCols);
+    }
+}
+
+// ------------------------------------------------------------------ host side
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn get_encode_fn()
+{
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(ptr);
+    });
+    return fn;
+}
+
+// 2-D map over a row-major [rows, cols] matrix with 128-byte rows per box
+// and the 128-byte swizzle; box = box_rows x (128 bytes).
+static bool make_map(CUtensorMap *m, const void *base, bool u8, uint64_t rows, uint64_t cols,
+                     uint32_t box_rows)
+{
+    EncodeTiledFn fn = get_encode_fn();
+    if (!fn) return false;
+    const uint32_t esz = u8 ? 1 : 2;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {cols * esz};
+    cuuint32_t box[2] = {128 / esz, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(m, u8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                    const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+static int sm_count()
+{
+    static int n = 0;
+    if (n == 0) {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+        if (n <= 0) n = 148;
+        if (n > kMaxCtas) n = kMaxCtas;
+    }
+    return n;
+}
+
+template <int kMode, bool kSwap, bool kFp8, int kBN>
+static cudaError_t run_gemm(const moe_shape_t &s, const GemmArgs &a, cudaStream_t st, int *host_err)
+{
+    using Cf = Cfg<kMode, kSwap, kFp8, kBN>;
+    auto kern = grouped_gemm_kernel<kMode, kSwap, kFp8, kBN>;
+    static std::once_flag once;
+    std::call_once(once, [&] {
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cf::kDynSmem);
+    });
+    const int Et = s.E + s.n_shared;
+    const bool u8 = kFp8;
+    const int K = kMode == 0 ? s.H : s.I;
+    const uint64_t w_rows = kMode == 0 ? 2ull * s.I : static_cast<uint64_t>(s.H);
+    // weight box rows: Swap-AB gate/up halves (64) or W2 rows (128); normal
+    // gate/up halves (128) or W2 rows (256)
+    const uint32_t wbox = kSwap ? (kMode == 0 ? 64 : 128) : (kMode == 0 ? 128 : 256);
+    const uint32_t xbox = kSwap ? kBN : 128;
+    CUtensorMap tm_w, tm_x;
+    if (!make_map(&tm_w, a.wgt, u8, Et * w_rows, K, wbox) ||
+        !make_map(&tm_x, a.act, u8, a.max_rows, K, xbox)) {
+        *host_err = MOE_ERR_CUDA;
+        return cudaSuccess;
+    }
+    GemmParams p;
+    p.offsets = a.offsets;
+    p.E_tot = Et;
+    p.K = K;
+    p.n_feat = kMode == 0 ? s.I : s.H;
+    p.w_rows = static_cast<int>(w_rows);
+    p.out_ld = kMode == 0 ? s.I : s.H;
+    p.out = a.out;
+    p.wscale = a.wscale;
+    p.ascale = a.ascale;
+    p.qscale = a.qscale;
+    p.status = a.status;
+    p.counters = a.counters;
+    p.partials = a.partials;
+    p.stream_k = 1;
+    cudaError_t err = cudaMemsetAsync(a.counters, 0, 2 * kMaxCtas * sizeof(int32_t), st);
+    if (err != cudaSuccess) return err;
+    kern<<<sm_count(), 192, Cf::kDynSmem, st>>>(tm_w, tm_x, p);
+    return cudaGetLastError();
+}
+
+int gemm_acc_cols(const GemmPlan &p) { return p.swap ? p.bn : 256; }
+
+cudaError_t launch_grouped_gemm(const moe_shape_t &s, const GemmPlan &p, const GemmArgs &a,
+                                cudaStream_t st, int *launches, int *host_err)
+{
+    *host_err = MOE_OK;
+    const bool fp8 = s.adtype == MOE_E4M3;
+    cudaError_t err = cudaSuccess;
+#define MOE_G(MODE, SWAP, FP8, BN) err = run_gemm<MODE, SWAP, FP8, BN>(s, a, st, host_err)
+#define MOE_BY_BN(MODE, FP8)                      \
+    switch (p.bn) {                               \
+    case 16: MOE_G(MODE, true, FP8, 16); break;   \
+    case 32: MOE_G(MODE, true, FP8, 32); break;   \
+    case 64: MOE_G(MODE, true, FP8, 64); break;   \
+    case 128: MOE_G(MODE, true, FP8, 128); break; \
+    default: MOE_G(MODE, true, FP8, 256); break;  \
+    }
+    if (p.swap) {
+        if (a.mode == 0) {
+            if (fp8) { MOE_BY_BN(0, true) } else { MOE_BY_BN(0, false) }
+        } else {
+            if (fp8) { MOE_BY_BN(1, true) } else { MOE_BY_BN(1, false) }
+        }
+    } else {
+        if (a.mode == 0) {
+            if (fp8) MOE_G(0, false, true, 256);
+            else MOE_G(0, false, false, 256);
+        } else {
+            if (fp8) MOE_G(1, false, true, 256);
+            else MOE_G(1, false, false, 256);
+        }
+    }
+#undef MOE_BY_BN
+#undef MOE_G
+    *launches += 1;
+    return err;
+}
+
+}  // namespace moe

@@ -1,0 +1,387 @@
+// small_kernels.cu - the memory-bound steps of the fused-MoE layer:
+//   routing (top-k gating), alignment/permutation, gather (+E4M3 quantisation)
+//   and the weighted combine.
+// The AWS post ("Mixture-of-Experts kernel engineering on Amazon SageMaker AI",
+// abstract) names these steps as token routing, data shuffling and expert
+// aggregation; the Chinese retelling (section "2. 用于FP8量化的Triton后端路由")
+// stresses keeping routing decisions on the GPU, without host-side control
+// flow.  Nothing here reads a routing result on the host.
+#include <cuda_bf16.h>
+#include <cuda_fp8.h>
+
+#include "common.cuh"
+
+namespace moe {
+
+// ------------------------------------------------------------------ routing
+// Order-preserving map of a float logit to an unsigned key: larger logit ->
+// larger key, -0 == +0, NaN below -inf (key 0).
+__device__ __forceinline__ uint32_t logit_key(float v)
+{
+    if (v != v) return 0u;
+    if (v == 0.0f) v = 0.0f;
+    uint32_t u = __float_as_uint(v);
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+__device__ __forceinline__ float warp_sum(float v)
+{
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+__device__ __forceinline__ float warp_max(float v)
+{
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+
+// One warp per token.  Lane l holds logits l, l+32, ...; the k winners are
+// found by k rounds of a warp-wide arg-max over the 64-bit key
+// (logit key, ~expert id): larger logit first, ties to the lower id.
+template <int kSlots>
+__global__ void __launch_bounds__(256) route_topk_kernel(const float *__restrict__ logits, int T,
+                                                         int E, int k, int gate, int renorm,
+                                                         float routed_scale, int32_t *ids,
+                                                         float *w)
+{
+    const int lane = threadIdx.x & 31;
+    const int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    if (t >= T) return;
+    const float *l = logits + static_cast<size_t>(t) * E;
+    uint64_t key[kSlots];
+    uint32_t taken = 0;
+#pragma unroll
+    for (int i = 0; i < kSlots; ++i) {
+        const int e = i * 32 + lane;
+        if (e < E) {
+            key[i] = (static_cast<uint64_t>(logit_key(l[e])) << 32) | (0xFFFFFFFFu - static_cast<uint32_t>(e));
+        } else {
+            key[i] = 0;
+            taken |= 1u << i;
+        }
+    }
+    int my_id = -1;
+    for (int j = 0; j < k; ++j) {
+        uint64_t best = 0;
+#pragma unroll
+        for (int i = 0; i < kSlots; ++i)
+            if (!((taken >> i) & 1u) && key[i] > best) best = key[i];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            const uint64_t other = __shfl_xor_sync(0xffffffffu, best, o);
+            best = other > best ? other : best;
+        }
+        const int id = static_cast<int>(0xFFFFFFFFu - static_cast<uint32_t>(best & 0xFFFFFFFFu));
+        if ((id & 31) == lane) taken |= 1u << (id >> 5);
+        if (lane == j) my_id = id;
+    }
+    const bool mine = lane < k;
+    const float v = mine ? l[my_id] : 0.0f;
+    float wt;
+    if (gate == MOE_GATE_SOFTMAX) {
+        if (renorm) {
+            const float m = __shfl_sync(0xffffffffu, v, 0);
+            const float ex = mine ? expf(v - m) : 0.0f;
+            wt = ex / warp_sum(ex);
+        } else {
+            float m = -INFINITY;
+            for (int e = lane; e < E; e += 32) m = fmaxf(m, l[e]);
+            m = warp_max(m);
+            float z = 0.0f;
+            for (int e = lane; e < E; e += 32) z += expf(l[e] - m);
+            z = warp_sum(z);
+            wt = expf(v - m) / z;
+        }
+    } else {
+        const float s = mine ? 1.0f / (1.0f + expf(-v)) : 0.0f;
+        wt = renorm ? s / warp_sum(s) : s;
+    }
+    if (mine) {
+        ids[static_cast<size_t>(t) * k + lane] = my_id;
+        w[static_cast<size_t>(t) * k + lane] = wt * routed_scale;
+    }
+}
+
+cudaError_t launch_route(const moe_shape_t &s, const float *logits, int32_t *ids, float *w,
+                         cudaStream_t st)
+{
+    const int threads = 256, blocks = (s.T * 32 + threads - 1) / threads;
+    const int slots = (s.E + 31) / 32;
+#define MOE_ROUTE(N)                                                                          \
+    route_topk_kernel<N><<<blocks, threads, 0, st>>>(logits, s.T, s.E, s.k, s.gate, s.renorm, \
+                                                     s.routed_scale, ids, w)
+    if (slots <= 1) MOE_ROUTE(1);
+    else if (slots <= 2) MOE_ROUTE(2);
+    else if (slots <= 4) MOE_ROUTE(4);
+    else if (slots <= 8) MOE_ROUTE(8);
+    else MOE_ROUTE(16);
+#undef MOE_ROUTE
+    return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------ align
+// Block b counts the expert ids of routed rows [b*1024, (b+1)*1024) into a
+// shared histogram (integer atomics: the counts do not depend on order).  The
+// last block to finish (ticket) turns the per-block histograms into counts,
+// padded segment offsets and each block's first slot per expert, fills pad
+// slots with -1 and writes the shared experts' rows.
+__global__ void __launch_bounds__(1024) align_count_kernel(
+    const int32_t *__restrict__ ids, int R, int T, int E, int n_shared, int pad,
+    int32_t *chunk_hist, int32_t *chunk_base, int32_t *counts, int32_t *offsets,
+    int32_t *sorted_rows, Ctrl *ctrl)
+{
+    extern __shared__ int32_t sh[];
+    __shared__ int s_last;
+    const int Et = E + n_shared;
+    const int tid = threadIdx.x, nb = gridDim.x;
+    for (int i = tid; i < Et; i += blockDim.x) sh[i] = 0;
+    __syncthreads();
+    const int f = blockIdx.x * kAlignChunk + tid;
+    if (f < R) {
+        const int e = ids[f];
+        if (e >= 0 && e < E) atomicAdd(&sh[e], 1);
+        else set_status(&ctrl->status, MOE_ERR_DEVICE_CHECK);
+    }
+    __syncthreads();
+    for (int i = tid; i < Et; i += blockDim.x) chunk_hist[static_cast<size_t>(blockIdx.x) * Et + i] = sh[i];
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) s_last = (atomicAdd(&ctrl->ticket, 1) == nb - 1);
+    __syncthreads();
+    if (!s_last) return;
+    __threadfence();
+    // totals and padded sizes
+    for (int e = tid; e < Et; e += blockDim.x) {
+        int c = 0;
+        if (e < E)
+            for (int b = 0; b < nb; ++b) c += __ldcg(&chunk_hist[static_cast<size_t>(b) * Et + e]);
+        else
+            c = T;
+        counts[e] = c;
+        sh[e] = (c + pad - 1) / pad * pad;
+    }
+    __syncthreads();
+    // exclusive scan of the padded sizes by warp 0 (contiguous chunk per lane)
+    if (tid < 32) {
+        const int per = (Et + 31) / 32;
+        const int lo = min(Et, tid * per), hi = min(Et, lo + per);
+        int sum = 0;
+        for (int e = lo; e < hi; ++e) sum += sh[e];
+        int inc = sum;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(0xffffffffu, inc, o);
+            if (tid >= o) inc += v;
+        }
+        int run = inc - sum;
+        for (int e = lo; e < hi; ++e) {
+            const int sz = sh[e];
+            offsets[e] = run;
+            sh[e] = run;
+            run += sz;
+        }
+        if (tid == 31) offsets[Et] = inc;
+    }
+    __syncthreads();
+    // first slot of each (block, expert) pair, pad slots, shared experts
+    for (int e = tid; e < Et; e += blockDim.x) {
+        const int start = sh[e];
+        if (e < E) {
+            int base = start;
+            for (int b = 0; b < nb; ++b) {
+                chunk_base[static_cast<size_t>(b) * Et + e] = base;
+                base += __ldcg(&chunk_hist[static_cast<size_t>(b) * Et + e]);
+            }
+        }
+        const int c = counts[e];
+        const int end = start + (c + pad - 1) / pad * pad;
+        for (int q = start + c; q < end; ++q) sorted_rows[q] = -1;
+    }
+    for (int s = 0; s < n_shared; ++s)
+        for (int t = tid; t < T; t += blockDim.x) sorted_rows[sh[E + s] + t] = R + s * T + t;
+    if (tid == 0) ctrl->ticket = 0;
+}
+
+// Each block places its 1024 routed rows: rank within the warp by
+// __match_any_sync, ranks of earlier warps by a prefix over per-warp counts,
+// plus the block's first slot for that expert.  The result is the stable
+// (ascending row index) order within every expert, independent of timing.
+__global__ void __launch_bounds__(1024) align_scatter_kernel(const int32_t *__restrict__ ids,
+                                                             int R, int E, int Et,
+                                                             const int32_t *chunk_base,
+                                                             int32_t *sorted_rows, int32_t *inv)
+{
+    extern __shared__ int32_t wc[];   // [32 warps][Et]
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    for (int i = tid; i < 32 * Et; i += blockDim.x) wc[i] = 0;
+    __syncthreads();
+    const int f = blockIdx.x * kAlignChunk + tid;
+    int e = f < R ? ids[f] : -1;
+    const bool valid = e >= 0 && e < E;
+    if (!valid) e = -1;
+    const unsigned same = __match_any_sync(0xffffffffu, e);
+    const int rank = __popc(same & ((1u << lane) - 1u));
+    if (valid && rank == 0) wc[warp * Et + e] = __popc(same);
+    __syncthreads();
+    for (int x = tid; x < Et; x += blockDim.x) {
+        int run = 0;
+        for (int q = 0; q < 32; ++q) {
+            const int c = wc[q * Et + x];
+            wc[q * Et + x] = run;
+            run += c;
+        }
+    }
+    __syncthreads();
+    if (f < R) {
+        if (valid) {
+            const int slot = chunk_base[static_cast<size_t>(blockIdx.x) * Et + e] + wc[warp * Et + e] + rank;
+            sorted_rows[slot] = f;
+            inv[f] = slot;
+        } else {
+            inv[f] = -1;
+        }
+    }
+}
+
+cudaError_t launch_align(const moe_shape_t &s, const int32_t *ids, int32_t *counts,
+                         int32_t *offsets, int32_t *sorted_rows, int32_t *inv, int32_t *chunk_hist,
+                         int32_t *chunk_base, Ctrl *ctrl, cudaStream_t st, int *launches)
+{
+    const int R = s.T * s.k, Et = s.E + s.n_shared;
+    const int nb = (R + kAlignChunk - 1) / kAlignChunk;
+    static bool attr_done = false;
+    if (!attr_done) {
+        cudaFuncSetAttribute(align_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             32 * kMaxExpertsTotal * 4);
+        attr_done = true;
+    }
+    cudaError_t err = cudaMemsetAsync(&ctrl->ticket, 0, sizeof(int32_t), st);
+    if (err != cudaSuccess) return err;
+    align_count_kernel<<<nb, kAlignChunk, Et * sizeof(int32_t), st>>>(
+        ids, R, s.T, s.E, s.n_shared, s.pad, chunk_hist, chunk_base, counts, offsets, sorted_rows, ctrl);
+    align_scatter_kernel<<<nb, kAlignChunk, 32 * Et * sizeof(int32_t), st>>>(ids, R, s.E, Et, chunk_base,
+                                                                             sorted_rows, inv);
+    *launches += 2;
+    return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------ gather
+// One warp per slot of the permuted buffer, 16-byte vectors along the row.
+template <bool kQuant>
+__global__ void __launch_bounds__(256) gather_kernel(const uint4 *__restrict__ x,
+                                                     const int32_t *__restrict__ sorted_rows,
+                                                     const int32_t *__restrict__ offsets, int Et,
+                                                     int T, int k, int H, float a1, void *xp)
+{
+    const int lane = threadIdx.x & 31;
+    const int nvec = H / 8;                       // 8 bf16 per 16 bytes
+    const int total = offsets[Et];
+    const int R = T * k;
+    for (int s = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; s < total;
+         s += (gridDim.x * blockDim.x) >> 5) {
+        const int f = sorted_rows[s];
+        const int t = f < 0 ? -1 : (f < R ? f / k : (f - R) % T);
+        if (!kQuant) {
+            uint4 *dst = reinterpret_cast<uint4 *>(xp) + static_cast<size_t>(s) * nvec;
+            const uint4 *src = x + static_cast<size_t>(t < 0 ? 0 : t) * nvec;
+            for (int v = lane; v < nvec; v += 32) dst[v] = t < 0 ? make_uint4(0, 0, 0, 0) : __ldg(src + v);
+        } else {
+            uint2 *dst = reinterpret_cast<uint2 *>(xp) + static_cast<size_t>(s) * nvec;
+            const uint4 *src = x + static_cast<size_t>(t < 0 ? 0 : t) * nvec;
+            for (int v = lane; v < nvec; v += 32) {
+                if (t < 0) {
+                    dst[v] = make_uint2(0, 0);
+                    continue;
+                }
+                const uint4 d = __ldg(src + v);
+                const uint32_t wv[4] = {d.x, d.y, d.z, d.w};
+                uint32_t q[2] = {0, 0};
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const uint32_t bits = (wv[i >> 1] >> ((i & 1) * 16)) & 0xFFFFu;
+                    const float val = __uint_as_float(bits << 16) / a1;
+                    const uint32_t c = __nv_cvt_float_to_fp8(val, __NV_SATFINITE, __NV_E4M3);
+                    q[i >> 2] |= (c & 0xFFu) << ((i & 3) * 8);
+                }
+                dst[v] = make_uint2(q[0], q[1]);
+            }
+        }
+    }
+}
+
+cudaError_t launch_gather(const moe_shape_t &s, const void *x, const int32_t *sorted_rows,
+                          const int32_t *offsets, float a1, void *xp, int64_t max_rows,
+                          cudaStream_t st)
+{
+    const int Et = s.E + s.n_shared;
+    const int64_t warps = max_rows;
+    int blocks = static_cast<int>((warps + 7) / 8);
+    if (blocks > 148 * 16) blocks = 148 * 16;
+    if (blocks < 1) blocks = 1;
+    if (s.adtype == MOE_E4M3)
+        gather_kernel<true><<<blocks, 256, 0, st>>>(static_cast<const uint4 *>(x), sorted_rows, offsets,
+                                                    Et, s.T, s.k, s.H, a1, xp);
+    else
+        gather_kernel<false><<<blocks, 256, 0, st>>>(static_cast<const uint4 *>(x), sorted_rows,
+                                                     offsets, Et, s.T, s.k, s.H, a1, xp);
+    return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------ combine
+// One block per token; each thread owns 4 consecutive outputs and sums the
+// k routed rows (weighted) then the shared rows, in that fixed order.
+__global__ void __launch_bounds__(256) combine_kernel(const float4 *__restrict__ y,
+                                                      const float *__restrict__ w,
+                                                      const int32_t *__restrict__ inv,
+                                                      const int32_t *__restrict__ offsets, int H,
+                                                      int k, int E, int n_shared, uint2 *out)
+{
+    const int t = blockIdx.x;
+    const int n4 = H / 4;
+    __shared__ int s_slot[kMaxTopK + 1];
+    __shared__ float s_w[kMaxTopK];
+    if (threadIdx.x < k) {
+        s_slot[threadIdx.x] = inv[static_cast<size_t>(t) * k + threadIdx.x];
+        s_w[threadIdx.x] = w[static_cast<size_t>(t) * k + threadIdx.x];
+    }
+    __syncthreads();
+    for (int c = threadIdx.x; c < n4; c += blockDim.x) {
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int j = 0; j < k; ++j) {
+            const int slot = s_slot[j];
+            if (slot < 0) continue;
+            const float wt = s_w[j];
+            const float4 v = __ldg(y + static_cast<size_t>(slot) * n4 + c);
+            acc.x = fmaf(wt, v.x, acc.x);
+            acc.y = fmaf(wt, v.y, acc.y);
+            acc.z = fmaf(wt, v.z, acc.z);
+            acc.w = fmaf(wt, v.w, acc.w);
+        }
+        for (int s = 0; s < n_shared; ++s) {
+            const float4 v = __ldg(y + static_cast<size_t>(offsets[E + s] + t) * n4 + c);
+            acc.x += v.x;
+            acc.y += v.y;
+            acc.z += v.z;
+            acc.w += v.w;
+        }
+        const __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y);
+        const __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z, acc.w);
+        uint2 o;
+        o.x = *reinterpret_cast<const uint32_t *>(&lo);
+        o.y = *reinterpret_cast<const uint32_t *>(&hi);
+        out[static_cast<size_t>(t) * n4 + c] = o;
+    }
+}
+
+cudaError_t launch_combine(const moe_shape_t &s, const float *y, const float *w,
+                           const int32_t *inv, const int32_t *offsets, void *out, cudaStream_t st)
+{
+    combine_kernel<<<s.T, 256, 0, st>>>(reinterpret_cast<const float4 *>(y), w, inv, offsets, s.H,
+                                        s.k, s.E, s.n_shared, static_cast<uint2 *>(out));
+    return cudaGetLastError();
+}
+
+}  // namespace moe
