@@ -210,10 +210,10 @@ def test_grouped_gemm_swiglu_matches_oracle(case):
     if fp8:
         got = orc.e4m3_decode(hv.ravel()).reshape(total, I) * a2
         refq = orc.e4m3_decode(orc.e4m3_encode(ref / a2).ravel()).reshape(total, I) * a2
-        assert rel_err(got, refq) <= FP8_TOL
+        assert rel_err(got, refq, "e4m3") <= FP8_TOL
     else:
         got = bf16_to_f64(hv.view(np.uint16))
-        assert rel_err(got, ref) <= BF16_TOL
+        assert rel_err(got, ref, "bf16") <= BF16_TOL
 
 
 @pytest.mark.parametrize("case", GEMM_CASES, ids=lambda c: c[0])
@@ -254,7 +254,7 @@ def test_combine_matches_oracle():
                 torch.from_numpy(o).cuda(), out)
     ref = orc.combine(y.astype(np.float64), w.astype(np.float64), v, o, E, ns)
     got = bf16_to_f64(host_bf16_bits(out))
-    assert rel_err(got, ref) <= 5e-3
+    assert rel_err(got, ref, "bf16") <= 1e-3
 
 
 # ------------------------------------------------------------------ the fused layer
@@ -267,11 +267,11 @@ def test_fused_tiny_all_tokens_both_variants_and_determinism():
         L = Layer(wl, d, variant=variant)
         got = L.run()
         assert L.status() == 0
-        assert rel_err(got, ref) <= BF16_TOL, variant
+        assert rel_err(got, ref, "bf16") <= BF16_TOL, variant
         outs.append(got)
         again = L.run()
         assert np.array_equal(got, again)          # bit-identical rerun
-    assert rel_err(outs[0], outs[1]) <= 5e-3       # Swap-AB == normal up to summation order
+    assert rel_err(outs[0], outs[1], "bf16") <= 2e-2       # Swap-AB == normal up to summation order
 
 
 @pytest.mark.parametrize("T", [1, 8, 64])
@@ -283,7 +283,7 @@ def test_fused_mixtral_decode_sampled(T):
     assert L.status() == 0
     toks = np.unique(np.linspace(0, T - 1, min(T, 6)).astype(np.int32))
     ref = oracle_forward(wl, d, tokens=toks)
-    assert rel_err(got[toks], ref) <= BF16_TOL
+    assert rel_err(got[toks], ref, "bf16") <= BF16_TOL
 
 
 def test_swap_ab_page_example_shape():
@@ -294,7 +294,7 @@ def test_swap_ab_page_example_shape():
     ref = oracle_forward(wl, d)
     for variant in (moe.SWAP_AB, moe.NORMAL):
         got = Layer(wl, d, variant=variant).run()
-        assert rel_err(got, ref) <= BF16_TOL
+        assert rel_err(got, ref, "bf16") <= BF16_TOL
 
 
 EDGE = [
@@ -316,7 +316,7 @@ def test_fused_edge_cases(wl, pad):
         L = Layer(wl, d, pad=pad, variant=variant)
         got = L.run()
         assert L.status() == 0
-        assert rel_err(got, ref) <= BF16_TOL, (variant, pad)
+        assert rel_err(got, ref, "bf16") <= BF16_TOL, (variant, pad)
 
 
 def _fp8_small(T=300):
@@ -336,4 +336,4 @@ def test_fused_fp8_weights_and_activations(variant):
     L = Layer(wl, d, variant=variant, a2=a2)
     got = L.run()
     assert L.status() == 0
-    assert rel_err(got, ref) <= FP8_TOL
+    assert rel_err(got, ref, "bf16") <= FP8_TOL
