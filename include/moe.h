@@ -140,6 +140,30 @@ int moe_align_permute(const moe_shape_t *shape, const int32_t *ids, int32_t *cou
                       size_t ws_bytes, moe_stream_t stream);
 
 /*
+ * Step 2 without a workspace (no counterpart on the pages: an addition for
+ * callers that cannot allocate).  Some callers cannot provide the `ws` buffer
+ * the call above needs -- for example an engine whose device memory is all
+ * reserved by its own allocator at start-up, or a latency-critical loop that
+ * may not call cudaMalloc because it can synchronise the device.  This call
+ * computes exactly what moe_align_permute computes, but keeps its scratch
+ * (per-block histograms and control words, 262,912 bytes) in one fixed array
+ * inside the library, held on every GPU that loads the library until the
+ * process exits.  It allocates nothing.
+ *   Limits: T*k <= 65536 routed rows and E + n_shared <= 513 experts; larger
+ *   shapes return MOE_ERR_UNSUPPORTED before anything is launched.
+ *   status: optional device int32 (may be NULL) that receives the call's
+ *   device status (MOE_ERR_DEVICE_CHECK for an id outside 0..E-1).
+ *   The first call on a device looks up the array's device address
+ *   (cudaGetSymbolAddress) while that device is current; make that first call
+ *   before any stream capture.  All calls share the one array, so calls that
+ *   overlap on the GPU (different streams, or different host threads using
+ *   the same device) race and must be serialised by the caller.
+ */
+int moe_align_permute_noalloc(const moe_shape_t *shape, const int32_t *ids, int32_t *counts,
+                              int32_t *offsets, int32_t *sorted_rows, int32_t *inv,
+                              int32_t *status, moe_stream_t stream);
+
+/*
  * Step 3 - gather the tokens into expert order.
  *   x [T, H] bf16 in; xp [max_rows, H] out, slot s = x[token of sorted_rows[s]]
  *   (zeros for pad slots).  adtype == MOE_E4M3: xp holds E4M3 codes of

@@ -29,7 +29,7 @@ STATUS = {0: "MOE_OK", -1: "MOE_ERR_INVALID_ARG", -2: "MOE_ERR_UNSUPPORTED",
 EXPORTS = ["moe_max_rows", "moe_workspace_size", "moe_route_topk", "moe_align_permute", "moe_gather",
            "moe_grouped_gemm_swiglu", "moe_grouped_gemm_down", "moe_combine", "moe_fused_forward",
            "moe_get_device_status", "moe_reset_device_status", "moe_status_string",
-           "moe_last_launch_count"]
+           "moe_last_launch_count", "moe_align_permute_noalloc"]
 
 
 class MoeError(RuntimeError):
@@ -78,6 +78,7 @@ def lib() -> C.CDLL:
             "moe_reset_device_status": [P, P],
             "moe_status_string": [C.c_int],
             "moe_last_launch_count": [],
+            "moe_align_permute_noalloc": [S, P, P, P, P, P, P, P],
         }
         for name, args in sig.items():
             fn = getattr(L, name)
@@ -146,6 +147,15 @@ def align_permute(shape, ids, counts, offsets, sorted_rows, inv, ws, stream=None
     _check(lib().moe_align_permute(C.byref(shape), _ptr(ids), _ptr(counts), _ptr(offsets),
                                    _ptr(sorted_rows), _ptr(inv), _ptr(ws), ws.numel(), _stream(stream)),
            "moe_align_permute")
+
+
+def align_permute_noalloc(shape, ids, counts, offsets, sorted_rows, inv, status=None, stream=None):
+    """moe_align_permute without a workspace: for callers that cannot allocate
+    one (the library keeps the scratch in a fixed device array; calls that
+    overlap on the GPU race)."""
+    _check(lib().moe_align_permute_noalloc(C.byref(shape), _ptr(ids), _ptr(counts), _ptr(offsets),
+                                           _ptr(sorted_rows), _ptr(inv), _ptr(status), _stream(stream)),
+           "moe_align_permute_noalloc")
 
 
 def gather(shape, x, sorted_rows, offsets, a1, xp, stream=None):
