@@ -161,12 +161,31 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------- our arm
-def measured_peak_hbm():
+def measured_peaks():
+    """(hbm GB/s, bf16 TF/s burst, bf16 TF/s sustained, kind)."""
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
-            return float(json.load(f)["hbm_gbs"]), "measured"
+            m = json.load(f)
+        return float(m["hbm_gbs"]), float(m["bf16_tflops"]), float(m["bf16_tflops_sustained"]), "measured"
     except (OSError, KeyError, ValueError):
-        return 6650.0, "fallback"
+        return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+def static_hidden_scale(wl) -> float:
+    """The oracle-calibrated static E4M3 scale of h (tests/golden), else 1."""
+    if wl.adtype != syn.E4M3:
+        return 1.0
+    path = os.path.join(ROOT, "tests", "golden", f"{wl.name}_hidden_scale.json")
+    with open(path) as f:
+        return float(json.load(f)["a2"])
+
+
+def moe_plan_is_normal(shape) -> bool:
+    """The operand order the library picks for this shape (mirrors its rule:
+    Swap-AB for T <= 128 or E4M3 weights with bf16 activations)."""
+    if shape.variant:
+        return shape.variant == 2
+    return not (shape.T <= 128 or (shape.wdtype == 1 and shape.adtype == 0))
 
 
 def ours_main(args, wl):
@@ -196,7 +215,8 @@ def ours_main(args, wl):
     w2 = to_dev(d["w2"], u8=esz == 1)
     s13 = torch.from_numpy(d["w13_scale"]).to(dev) if esz == 1 else None
     s2 = torch.from_numpy(d["w2_scale"]).to(dev) if esz == 1 else None
-    a1, a2 = float(d["a1"]), float(args.a2)
+    a1 = float(d["a1"])
+    a2 = float(args.a2) if args.a2 is not None else static_hidden_scale(wl)
     out = torch.empty((wl.T, wl.H), dtype=torch.bfloat16, device=dev)
     ws = moe.workspace(shape, device=dev)
     stream = torch.cuda.current_stream(dev)
@@ -275,10 +295,24 @@ def ours_main(args, wl):
     aesz = 1 if wl.adtype else 2
     g1_bytes = w13_bytes + slots * wl.H * aesz + slots * wl.I * aesz
     g2_bytes = w2_bytes + slots * wl.I * aesz + slots * wl.H * 4
-    peak, peak_kind = measured_peak_hbm()
-    ach = g1_bytes / (t_g1 * 1e-3) / 1e9
+    hbm_peak, tc_burst, tc_sust, peak_kind = measured_peaks()
     layer_bytes = active * weight_bytes_per_expert(wl) + wl.T * wl.H * 2 * 2 + wl.T * wl.E * 4
-    flops = 2.0 * 3 * wl.H * wl.I * (wl.T * wl.k + wl.n_shared * wl.T)
+    real_rows = wl.T * wl.k + wl.n_shared * wl.T
+    flops = 2.0 * 3 * wl.H * wl.I * real_rows
+    g1_flops = 2.0 * 2 * wl.H * wl.I * real_rows
+    decode = not moe_plan_is_normal(shape)
+    if decode:
+        roof = {"bound": "hbm", "achieved": g1_bytes / (t_g1 * 1e-3) / 1e9, "peak": hbm_peak, "unit": "GB/s",
+                "algorithmic_bytes": g1_bytes}
+    else:
+        # a GEMM timed on its own runs at the burst clock; E4M3 doubles the bf16 rate
+        peak = tc_burst * (2.0 if wl.adtype == syn.E4M3 else 1.0)
+        roof = {"bound": "tensor", "achieved": g1_flops / (t_g1 * 1e-3) / 1e12, "peak": peak,
+                "unit": "TFLOP/s", "algorithmic_flops": g1_flops}
+    roof.update({"frac": roof["achieved"] / roof["peak"], "peak_kind": peak_kind, "traffic": None,
+                 "kernel": "grouped_gemm (gate/up + SwiGLU)", "ms": t_g1, "down_ms": t_g2,
+                 "down_gbs": g2_bytes / (t_g2 * 1e-3) / 1e9,
+                 "down_tflops": 2.0 * wl.H * wl.I * real_rows / (t_g2 * 1e-3) / 1e12})
 
     # end to end through the C ABI with host buffers: pinned H2D of x and
     # logits, the fused call, D2H of out, every step
@@ -320,10 +354,7 @@ def ours_main(args, wl):
         "data": "synthetic", "config": config_of(wl, f"replicas x{world}" if world > 1 else "1 GPU"),
         "hbm_gbs": layer_bytes / (ms_per_step * 1e-3) / 1e9, "tflops": flops / (ms_per_step * 1e-3) / 1e12,
         "active_experts": active,
-        "roofline": {"bound": "hbm", "kernel": "grouped_gemm (gate/up + SwiGLU)", "achieved": ach,
-                     "peak": peak, "peak_kind": peak_kind, "unit": "GB/s", "frac": ach / peak,
-                     "traffic": None, "algorithmic_bytes": g1_bytes, "ms": t_g1,
-                     "down_ms": t_g2, "down_gbs": g2_bytes / (t_g2 * 1e-3) / 1e9},
+        "roofline": roof,
         "e2e": {"value": e2e_val, "unit": UNIT, "h2d_bytes_per_step": int(hx.numel() * 2 + hl.numel() * 4),
                 "d2h_bytes_per_step": int(ho.numel() * 2)},
         "gpu_launches": launches_per_step * args.steps,
@@ -347,7 +378,9 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="mixtral_decode", choices=sorted(syn.WORKLOADS))
     ap.add_argument("--T", type=int, default=None)
-    ap.add_argument("--a2", type=float, default=1.0, help="static hidden-activation scale (FP8 activations)")
+    ap.add_argument("--E", type=int, default=None, help="override the routed expert count (small profiling cases)")
+    ap.add_argument("--a2", type=float, default=None,
+                    help="static hidden-activation scale (FP8 activations; default: the calibrated golden value)")
     ap.add_argument("--ref-budget", type=float, default=15.0, help="seconds of host time per oracle sample")
     ap.add_argument("--no-cpu", action="store_true", help="skip the cpu_baseline leg")
     args = ap.parse_args()
@@ -356,6 +389,9 @@ def main():
     wl = syn.WORKLOADS[args.workload]
     if args.T is not None:
         wl = wl.with_T(args.T)
+    if args.E is not None:
+        import dataclasses
+        wl = dataclasses.replace(wl, E=args.E, name=f"{wl.name}_E{args.E}")
     if args.impl == "reference":
         return reference_main(args, wl)
     return ours_main(args, wl)

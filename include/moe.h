@@ -89,9 +89,11 @@ enum { MOE_VARIANT_AUTO = 0, MOE_VARIANT_SWAP_AB = 1, MOE_VARIANT_NORMAL = 2 };
  *            rows in the tensor core's M slot and the tokens in N (the
  *            "Swap-AB" of the AWS post, B^T[N,K] x A^T[K,M] = C^T[N,M], used
  *            when an expert sees few rows); MOE_VARIANT_NORMAL puts token rows
- *            in M; MOE_VARIANT_AUTO picks Swap-AB when no expert can receive 64
- *            or more rows (T < 64), else normal.  Results are the same up to
- *            fp32 summation order.
+ *            in M; MOE_VARIANT_AUTO picks Swap-AB when no expert can receive more
+ *            than 128 rows (T <= 128; 128 is the fixed M extent of a one-SM
+ *            tcgen05.mma), else normal.  Results are the same up to fp32
+ *            summation order.  E4M3 weights with bf16 activations always
+ *            use Swap-AB.
  */
 typedef struct {
     int32_t T, H, I, E, k, n_shared;

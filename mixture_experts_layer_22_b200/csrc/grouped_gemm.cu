@@ -31,6 +31,7 @@
 // recompiled per batch size.
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_fp8.h>
 
 #include <mutex>
@@ -57,22 +58,35 @@ struct GemmParams {
     int stream_k;     // 0: whole tiles only
 };
 
-template <int kMode, bool kSwap, bool kFp8, int kBN>
+template <int kMode, bool kSwap, bool kFp8, int kBN, bool kW8 = false>
 struct Cfg {
     static constexpr int kStageA = 128 * 128;               // 128 rows x 128 bytes
     static constexpr int kStageB = kBN * 128;
     static constexpr int kStage = kStageA + kStageB;
     static constexpr int kDynBudget = 205 * 1024;
     static constexpr int kStagesRaw = kDynBudget / kStage;
-    static constexpr int kStages = kStagesRaw > 12 ? 12 : kStagesRaw;
-    static constexpr int kDynSmem = kStages * kStage + 1024;
+    static constexpr int kStagesFull = kStagesRaw > 12 ? 12 : kStagesRaw;
+    // E4M3 weights with bf16 activations (kW8): one smem stage holds a raw
+    // E4M3 weight tile (128 rows x 128 codes) and the bf16 activation rows of
+    // both K halves; the converted bf16 weight slabs (K = 64, 32 columns) go
+    // to tensor memory, from where the MMA reads its A operand.
+    static constexpr int kStageW8 = kStageA + 2 * kStageB;
+    static constexpr int kStagesW8Fit = kDynBudget / kStageW8;
+    static constexpr int kStagesW8 = kStagesW8Fit > 10 ? 10 : kStagesW8Fit;
+    static constexpr int kStages = kW8 ? kStagesW8 : kStagesFull;
+    static constexpr int kDynSmem = (kW8 ? kStagesW8 * kStageW8 : kStagesFull * kStage) + 1024;
+    static constexpr int kThreads = kW8 ? 448 : 192;
     static constexpr int kAccCols = kSwap ? kBN : 256;      // fp32 columns per accumulator
-    static constexpr int kTmemCols = (2 * kAccCols) <= 32 ? 32 : 2 * kAccCols;
+    static constexpr int kTmemCols = kW8 ? 512 : ((2 * kAccCols) <= 32 ? 32 : 2 * kAccCols);
+    static constexpr int kAColBase = 2 * kAccCols;                   // first TMEM column of the A slabs
+    static constexpr int kAStages = 8;                               // A slabs of 32 columns
     static constexpr int kRowsTile = kSwap ? kBN : 128;     // token rows per tile
     static constexpr int kFeatTile = kMode == 0 ? (kSwap ? 64 : 128) : (kSwap ? 128 : 256);
-    static constexpr int kKStage = kFp8 ? 128 : 64;         // elements per 128-byte row
+    static constexpr int kKStage = (kFp8 || kW8) ? 128 : 64;   // K elements per work step
     static constexpr uint32_t kFmt = kFp8 ? 0u : 1u;
-    static_assert(kStages >= 2, "smem ring too small");
+    static_assert(kW8 ? kStagesW8 >= 4 : kStagesFull >= 2, "smem ring too small");
+    static_assert(!kW8 || (kSwap && !kFp8 && kBN <= 128), "E4M3-weight/bf16-activation path: Swap-AB, BN <= 128");
+    static_assert(!kW8 || kAColBase + kAStages * 32 <= 512, "tensor memory for the A slabs");
     static_assert(kTmemCols <= 512, "tensor memory");
 };
 
@@ -191,12 +205,45 @@ __device__ __forceinline__ uint32_t e4m3_code(float v)
     return static_cast<uint32_t>(__nv_cvt_float_to_fp8(v, __NV_SATFINITE, __NV_E4M3)) & 0xFFu;
 }
 
-template <int kMode, bool kSwap, bool kFp8, int kBN>
-__global__ void __launch_bounds__(192, 1)
+// 64 E4M3 codes (four 16-byte chunks of one swizzled 128-byte row) -> 64
+// bf16 values packed two per 32-bit word, K order.  Exact: every E4M3 value
+// is an fp16 value and a bf16 value.
+__device__ __forceinline__ void e4m3x64_to_bf16(const uint8_t *row, int r, int half, uint32_t (&o)[32])
+{
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        const int c = 4 * half + q;
+        const uint4 v = *reinterpret_cast<const uint4 *>(row + ((c ^ (r & 7)) << 4));
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const uint16_t pair = static_cast<uint16_t>(w[i >> 1] >> ((i & 1) * 16));
+            const uint32_t h2 = cvt_e4m3x2_f16x2(pair);
+            const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&h2));
+            o[q * 8 + i] = pack_bf16x2(f.x, f.y);
+        }
+    }
+}
+
+// Wait (bounded, ignoring the abort flag) for the last `issued` fills of a
+// ring whose next stage/phase is (stage, phase): lets in-flight TMA copies
+// land before an aborting CTA exits.
+__device__ __forceinline__ void drain_ring(uint64_t *full, int nstages, int stage, uint32_t phase, int issued)
+{
+    for (int i = 0; i < nstages && i < issued; ++i) {
+        stage = stage == 0 ? nstages - 1 : stage - 1;
+        if (stage == nstages - 1) phase ^= 1u;
+        volatile int no_abort = 0;
+        mbar_wait(smem_u32(&full[stage]), phase, &no_abort);
+    }
+}
+
+template <int kMode, bool kSwap, bool kFp8, int kBN, bool kW8 = false>
+__global__ void __launch_bounds__(Cfg<kMode, kSwap, kFp8, kBN, kW8>::kThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tm_w,
                         const __grid_constant__ CUtensorMap tm_x, GemmParams p)
 {
-    using C = Cfg<kMode, kSwap, kFp8, kBN>;
+    using C = Cfg<kMode, kSwap, kFp8, kBN, kW8>;
     extern __shared__ uint8_t dyn_smem[];
     __shared__ int s_off[kMaxExpertsTotal + 1];
     __shared__ int s_prefix[kMaxExpertsTotal + 1];
@@ -206,6 +253,8 @@ __global__ void __launch_bounds__(192, 1)
     __shared__ volatile int s_abort;
     __shared__ int s_is_last;
     __shared__ float s_xchg[kMode == 0 && kSwap ? 16 * 64 : 1];
+    constexpr int kAN = kW8 ? C::kAStages : 1;
+    __shared__ __align__(8) uint64_t s_a_full[kAN], s_a_empty[kAN];
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int Et = p.E_tot;
@@ -217,13 +266,21 @@ __global__ void __launch_bounds__(192, 1)
         s_abort = 0;
         for (int i = 0; i < C::kStages; ++i) {
             mbar_init(smem_u32(&s_full[i]), 1);
-            mbar_init(smem_u32(&s_empty[i]), 1);
+            // kW8: the stage is free once the 8 converter warps have read the
+            // raw tile and the MMA has read the activations (one commit)
+            mbar_init(smem_u32(&s_empty[i]), kW8 ? 9 : 1);
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(smem_u32(&s_tfull[i]), 1);
             mbar_init(smem_u32(&s_tempty[i]), 4);
         }
         mbar_init(smem_u32(&s_drain), 1);
+        if (kW8) {
+            for (int i = 0; i < kAN; ++i) {
+                mbar_init(smem_u32(&s_a_full[i]), 4);         // the four warps of one K half
+                mbar_init(smem_u32(&s_a_empty[i]), 1);
+            }
+        }
         fence_mbar_init();
         prefetch_tmap(&tm_w);
         prefetch_tmap(&tm_x);
@@ -279,7 +336,150 @@ __global__ void __launch_bounds__(192, 1)
     S.sk_total = static_cast<long long>(S.sk_tiles) * S.KT;
     S.sk_ctas = static_cast<int>(S.sk_total < S.G ? S.sk_total : S.G);
 
-    if (warp == 0) {
+
+    if (kW8 && warp == 0) {
+        // ================= TMA producer (E4M3 weights, bf16 activations) ====
+        if (lane == 0) {
+            const uint64_t pol_w = policy_evict_first();
+            const uint64_t pol_x = policy_evict_last();
+            int stage = 0, in_flight = 0;
+            uint32_t phase = 0;
+            ItemIter I;
+            iter_init(I, S, blockIdx.x);
+            Item it;
+            bool ok = true;
+            while (ok && iter_next<C::kRowsTile>(I, S, s_prefix, s_off, Et, n_ft, it)) {
+                const int row0 = s_off[it.e] + it.rt * C::kRowsTile;
+                const int rows = min(C::kRowsTile, s_off[it.e + 1] - row0);
+                const int wbase = it.e * p.w_rows;
+                for (int kk = it.kb; kk < it.ke; ++kk) {
+                    if (!mbar_wait(smem_u32(&s_empty[stage]), phase ^ 1u, &s_abort)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t fb = smem_u32(&s_full[stage]);
+                    mbar_arrive_expect_tx(fb, C::kStageA + 2 * rows * 128);
+                    const uint32_t sa = smem_u32(tiles + stage * C::kStageW8);
+                    const int kx8 = kk * 128;                      // E4M3 elements
+                    if (kMode == 0) {
+                        tma_load_2d(sa, &tm_w, fb, kx8, wbase + it.ft * 64, pol_w);
+                        tma_load_2d(sa + 64 * 128, &tm_w, fb, kx8, wbase + p.n_feat + it.ft * 64, pol_w);
+                    } else {
+                        tma_load_2d(sa, &tm_w, fb, kx8, wbase + it.ft * 128, pol_w);
+                    }
+                    for (int hh = 0; hh < 2; ++hh)
+                        for (int rr = 0; rr < rows; rr += 16)
+                            tma_load_2d(sa + C::kStageA + hh * C::kStageB + rr * 128, &tm_x, fb,
+                                        kk * 128 + hh * 64, row0 + rr, pol_x);
+                    ++in_flight;
+                    if (++stage == C::kStages) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+            if (!ok) drain_ring(s_full, C::kStages, stage, phase, in_flight);
+        }
+    } else if (kW8 && warp >= 6) {
+        // ================= E4M3 -> bf16 converters (warps 6..13) ============
+        // Warp w converts K half (w - 6) / 4 of each stage for the 32 weight
+        // rows of its tensor-memory lane quarter (w % 4): thread = one row,
+        // 64 codes -> 32 packed columns, stored into an A slab with tcgen05.st.
+        const int half = (warp - 6) >> 2;
+        const int q = warp & 3;
+        const int r = q * 32 + lane;
+        const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
+        int stage = 0, j = 0;
+        uint32_t phase = 0;
+        ItemIter I;
+        iter_init(I, S, blockIdx.x);
+        Item it;
+        bool ok = true;
+        while (ok && iter_next<C::kRowsTile>(I, S, s_prefix, s_off, Et, n_ft, it)) {
+            for (int kk = it.kb; kk < it.ke; ++kk, ++j) {
+                // half-step 2j + half uses slab (2j + half) % kAStages
+                const int qs = 2 * j + half;
+                const int as = qs % C::kAStages;
+                const uint32_t aph = static_cast<uint32_t>(qs / C::kAStages) & 1u;
+                if (!mbar_wait(smem_u32(&s_full[stage]), phase, &s_abort) ||
+                    !mbar_wait(smem_u32(&s_a_empty[as]), aph ^ 1u, &s_abort)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                uint32_t o[32];
+                e4m3x64_to_bf16(tiles + stage * C::kStageW8 + r * 128, r, half, o);
+                tmem_st32(tmem_base + lane_base + C::kAColBase + as * 32, o);
+                tmem_wait_st();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) {
+                    mbar_arrive(smem_u32(&s_a_full[as]));
+                    mbar_arrive(smem_u32(&s_empty[stage]));
+                }
+                if (++stage == C::kStages) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
+        }
+    } else if (kW8 && warp == 1) {
+        // ================= MMA issuer (A = bf16 slabs in TMEM, B = smem) ====
+        if (lane == 0) {
+            int stage = 0, acc = 0, qs = 0;
+            uint32_t phase = 0, acc_phase = 0;
+            ItemIter I;
+            iter_init(I, S, blockIdx.x);
+            Item it;
+            bool ok = true;
+            while (ok && iter_next<C::kRowsTile>(I, S, s_prefix, s_off, Et, n_ft, it)) {
+                if (!mbar_wait(smem_u32(&s_tempty[acc]), acc_phase ^ 1u, &s_abort)) break;
+                tc_fence_after();
+                const uint32_t d = tmem_base + acc * C::kAccCols;
+                const int seg = s_off[it.e + 1] - s_off[it.e];
+                const int n = min(C::kRowsTile, seg - it.rt * C::kRowsTile);
+                const uint32_t idesc = idesc_make(1u, 128, n);
+                for (int kk = it.kb; ok && kk < it.ke; ++kk) {
+                    if (!mbar_wait(smem_u32(&s_full[stage]), phase, &s_abort)) {
+                        ok = false;
+                        break;
+                    }
+                    for (int hh = 0; hh < 2; ++hh, ++qs) {
+                        const int as = qs % C::kAStages;
+                        const uint32_t aph = static_cast<uint32_t>(qs / C::kAStages) & 1u;
+                        if (!mbar_wait(smem_u32(&s_a_full[as]), aph, &s_abort)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                        const uint32_t ta = tmem_base + C::kAColBase + as * 32;
+                        const uint32_t sb = smem_u32(tiles + stage * C::kStageW8 + C::kStageA + hh * C::kStageB);
+#pragma unroll
+                        for (int s4 = 0; s4 < 4; ++s4) {
+                            const uint32_t accum = (kk > it.kb || hh > 0 || s4 > 0) ? 1u : 0u;
+                            mma_bf16_tmem_a(d, ta + s4 * 8, sdesc_k_sw128(sb + s4 * 32), idesc, accum);
+                        }
+                        mma_commit(smem_u32(&s_a_empty[as]));
+                    }
+                    if (!ok) break;
+                    mma_commit(smem_u32(&s_empty[stage]));
+                    if (++stage == C::kStages) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                if (!ok) break;
+                mma_commit(smem_u32(&s_tfull[acc]));
+                if (++acc == 2) {
+                    acc = 0;
+                    acc_phase ^= 1u;
+                }
+            }
+            mma_commit(smem_u32(&s_drain));
+            volatile int no_abort = 0;
+            mbar_wait(smem_u32(&s_drain), 0, &no_abort);
+        }
+    } else if (!kW8 && warp == 0) {
         // ================= TMA producer =================
         if (lane == 0) {
             const uint64_t pol_w = policy_evict_first();
@@ -293,6 +493,7 @@ __global__ void __launch_bounds__(192, 1)
             bool ok = true;
             while (ok && iter_next<C::kRowsTile>(I, S, s_prefix, s_off, Et, n_ft, it)) {
                 const int row0 = s_off[it.e] + it.rt * C::kRowsTile;
+                const int rows = min(C::kRowsTile, s_off[it.e + 1] - row0);
                 const int wbase = it.e * p.w_rows;
                 for (int kk = it.kb; kk < it.ke; ++kk) {
                     if (!mbar_wait(smem_u32(&s_empty[stage]), phase ^ 1u, &s_abort)) {
@@ -300,7 +501,8 @@ __global__ void __launch_bounds__(192, 1)
                         break;
                     }
                     const uint32_t fb = smem_u32(&s_full[stage]);
-                    mbar_arrive_expect_tx(fb, C::kStage);
+                    // Swap-AB: only the tile's own token rows (16-row boxes)
+                    mbar_arrive_expect_tx(fb, kSwap ? C::kStageA + rows * 128 : C::kStage);
                     const uint32_t sa = smem_u32(tiles + stage * C::kStage);
                     const uint32_t sb = sa + C::kStageA;
                     const int kx = kk * C::kKStage;
@@ -311,7 +513,8 @@ __global__ void __launch_bounds__(192, 1)
                         } else {
                             tma_load_2d(sa, &tm_w, fb, kx, wbase + it.ft * 128, pol_w);
                         }
-                        tma_load_2d(sb, &tm_x, fb, kx, row0, pol_x);
+                        for (int rr = 0; rr < rows; rr += 16)
+                            tma_load_2d(sb + rr * 128, &tm_x, fb, kx, row0 + rr, pol_x);
                     } else {
                         tma_load_2d(sa, &tm_x, fb, kx, row0, pol_x);
                         if (kMode == 0) {
@@ -328,19 +531,9 @@ __global__ void __launch_bounds__(192, 1)
                     }
                 }
             }
-            if (!ok) {
-                // let copies already issued land before the CTA can exit
-                int st = stage;
-                uint32_t ph = phase;
-                for (int i = 0; i < C::kStages && i < in_flight; ++i) {
-                    st = st == 0 ? C::kStages - 1 : st - 1;
-                    if (st == C::kStages - 1) ph ^= 1u;
-                    volatile int no_abort = 0;
-                    mbar_wait(smem_u32(&s_full[st]), ph, &no_abort);
-                }
-            }
+            if (!ok) drain_ring(s_full, C::kStages, stage, phase, in_flight);   // let issued copies land
         }
-    } else if (warp == 1) {
+    } else if (!kW8 && warp == 1) {
         // ================= MMA issuer =================
         if (lane == 0) {
             int stage = 0;
@@ -395,7 +588,7 @@ __global__ void __launch_bounds__(192, 1)
             volatile int no_abort = 0;
             mbar_wait(smem_u32(&s_drain), 0, &no_abort);
         }
-    } else {
+    } else if (warp >= 2 && warp <= 5) {
         // ================= epilogue (warps 2..5) =================
         const int q = warp & 3;                 // tensor-memory lane quarter
         const int r = q * 32 + lane;            // accumulator row of this thread
@@ -656,25 +849,26 @@ static int sm_count()
     return n;
 }
 
-template <int kMode, bool kSwap, bool kFp8, int kBN>
+template <int kMode, bool kSwap, bool kFp8, int kBN, bool kW8 = false>
 static cudaError_t run_gemm(const moe_shape_t &s, const GemmArgs &a, cudaStream_t st, int *host_err)
 {
-    using Cf = Cfg<kMode, kSwap, kFp8, kBN>;
-    auto kern = grouped_gemm_kernel<kMode, kSwap, kFp8, kBN>;
+    using Cf = Cfg<kMode, kSwap, kFp8, kBN, kW8>;
+    auto kern = grouped_gemm_kernel<kMode, kSwap, kFp8, kBN, kW8>;
     static std::once_flag once;
     std::call_once(once, [&] {
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cf::kDynSmem);
     });
     const int Et = s.E + s.n_shared;
-    const bool u8 = kFp8;
+    const bool u8 = kFp8;              // activations are E4M3 codes
+    const bool u8w = kFp8 || kW8;      // weights are E4M3 codes
     const int K = kMode == 0 ? s.H : s.I;
     const uint64_t w_rows = kMode == 0 ? 2ull * s.I : static_cast<uint64_t>(s.H);
     // weight box rows: Swap-AB gate/up halves (64) or W2 rows (128); normal
     // gate/up halves (128) or W2 rows (256)
     const uint32_t wbox = kSwap ? (kMode == 0 ? 64 : 128) : (kMode == 0 ? 128 : 256);
-    const uint32_t xbox = kSwap ? kBN : 128;
+    const uint32_t xbox = kSwap ? 16 : 128;     // Swap-AB loads token rows in 16-row boxes
     CUtensorMap tm_w, tm_x;
-    if (!make_map(&tm_w, a.wgt, u8, Et * w_rows, K, wbox) ||
+    if (!make_map(&tm_w, a.wgt, u8w, Et * w_rows, K, wbox) ||
         !make_map(&tm_x, a.act, u8, a.max_rows, K, xbox)) {
         *host_err = MOE_ERR_CUDA;
         return cudaSuccess;
@@ -696,7 +890,7 @@ static cudaError_t run_gemm(const moe_shape_t &s, const GemmArgs &a, cudaStream_
     p.stream_k = 1;
     cudaError_t err = cudaMemsetAsync(a.counters, 0, 2 * kMaxCtas * sizeof(int32_t), st);
     if (err != cudaSuccess) return err;
-    kern<<<sm_count(), 192, Cf::kDynSmem, st>>>(tm_w, tm_x, p);
+    kern<<<sm_count(), Cf::kThreads, Cf::kDynSmem, st>>>(tm_w, tm_x, p);
     return cudaGetLastError();
 }
 
@@ -707,7 +901,23 @@ cudaError_t launch_grouped_gemm(const moe_shape_t &s, const GemmPlan &p, const G
 {
     *host_err = MOE_OK;
     const bool fp8 = s.adtype == MOE_E4M3;
+    const bool w8 = s.wdtype == MOE_E4M3 && s.adtype == MOE_BF16;
     cudaError_t err = cudaSuccess;
+    if (w8) {
+#define MOE_W8(MODE, BN) err = run_gemm<MODE, true, false, BN, true>(s, a, st, host_err)
+#define MOE_W8_BY_BN(MODE)                   \
+    switch (p.bn) {                          \
+    case 16: MOE_W8(MODE, 16); break;        \
+    case 32: MOE_W8(MODE, 32); break;        \
+    case 64: MOE_W8(MODE, 64); break;        \
+    default: MOE_W8(MODE, 128); break;       \
+    }
+        if (a.mode == 0) { MOE_W8_BY_BN(0) } else { MOE_W8_BY_BN(1) }
+#undef MOE_W8_BY_BN
+#undef MOE_W8
+        *launches += 1;
+        return err;
+    }
 #define MOE_G(MODE, SWAP, FP8, BN) err = run_gemm<MODE, SWAP, FP8, BN>(s, a, st, host_err)
 #define MOE_BY_BN(MODE, FP8)                      \
     switch (p.bn) {                               \

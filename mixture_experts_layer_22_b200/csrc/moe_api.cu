@@ -30,7 +30,6 @@ int validate_shape(const moe_shape_t *s, bool need_gemm)
     if (need_gemm) {
         if (s->H % 128 != 0 || s->I % 128 != 0) return MOE_ERR_UNSUPPORTED;
         if (s->pad % 16 != 0 || s->pad > 256) return MOE_ERR_UNSUPPORTED;
-        if (s->wdtype == MOE_E4M3 && s->adtype == MOE_BF16) return MOE_ERR_UNSUPPORTED;
     }
     return MOE_OK;
 }
@@ -40,11 +39,17 @@ GemmPlan plan_gemm(const moe_shape_t &s)
     GemmPlan p;
     // One tcgen05.mma on one SM has a fixed 128-row M extent: when no expert
     // can receive 128 rows or more, weights go to M and tokens to N.
-    p.swap = s.variant == MOE_VARIANT_SWAP_AB || (s.variant == MOE_VARIANT_AUTO && s.T <= 128);
+    // E4M3 weights with bf16 activations are converted in the weight (M)
+    // slot, so that path is always Swap-AB.
+    p.swap = s.variant == MOE_VARIANT_SWAP_AB || (s.variant == MOE_VARIANT_AUTO && s.T <= 128) ||
+             (s.wdtype == MOE_E4M3 && s.adtype == MOE_BF16);
     if (p.swap) {
         const int rows = (s.T + s.pad - 1) / s.pad * s.pad;   // worst case rows of one expert
         int bn = 16;
-        while (bn < rows && bn < 256) bn <<= 1;
+        // the E4M3-weight path keeps converted weight slabs in tensor memory
+        // next to the accumulators, which caps its token tile at 128 rows
+        const int cap = (s.wdtype == MOE_E4M3 && s.adtype == MOE_BF16) ? 128 : 256;
+        while (bn < rows && bn < cap) bn <<= 1;
         p.bn = bn;
     } else {
         p.bn = 256;

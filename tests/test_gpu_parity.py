@@ -173,41 +173,49 @@ def _segments(T, E, k, ns, pad, seed):
     return orc.align(ids, E, ns, pad)
 
 
-GEMM_CASES = [  # (name, T, H, I, E, k, ns, variant, fp8)
-    ("swap_tiny", 16, 256, 512, 8, 2, 0, moe.SWAP_AB, False),
-    ("normal_tiny", 16, 256, 512, 8, 2, 0, moe.NORMAL, False),
-    ("swap_decode", 64, 1024, 1024, 8, 2, 0, moe.SWAP_AB, False),
-    ("normal_prefill", 700, 512, 384, 6, 2, 0, moe.NORMAL, False),
-    ("swap_shared", 40, 256, 256, 16, 4, 1, moe.SWAP_AB, False),
-    ("swap_fp8", 64, 512, 512, 8, 2, 0, moe.SWAP_AB, True),
-    ("normal_fp8", 500, 512, 512, 8, 2, 0, moe.NORMAL, True),
+GEMM_CASES = [  # (name, T, H, I, E, k, ns, variant, weight dtype, activation dtype)
+    ("swap_tiny", 16, 256, 512, 8, 2, 0, moe.SWAP_AB, syn.BF16, syn.BF16),
+    ("normal_tiny", 16, 256, 512, 8, 2, 0, moe.NORMAL, syn.BF16, syn.BF16),
+    ("swap_decode", 64, 1024, 1024, 8, 2, 0, moe.SWAP_AB, syn.BF16, syn.BF16),
+    ("normal_prefill", 700, 512, 384, 6, 2, 0, moe.NORMAL, syn.BF16, syn.BF16),
+    ("swap_shared", 40, 256, 256, 16, 4, 1, moe.SWAP_AB, syn.BF16, syn.BF16),
+    ("swap_fp8", 64, 512, 512, 8, 2, 0, moe.SWAP_AB, syn.E4M3, syn.E4M3),
+    ("normal_fp8", 500, 512, 512, 8, 2, 0, moe.NORMAL, syn.E4M3, syn.E4M3),
+    ("w8a16_decode", 32, 1024, 512, 16, 8, 1, moe.AUTO, syn.E4M3, syn.BF16),
+    ("w8a16_t128", 128, 512, 256, 32, 8, 1, moe.AUTO, syn.E4M3, syn.BF16),
+    ("w8a16_t1", 1, 768, 384, 8, 4, 1, moe.AUTO, syn.E4M3, syn.BF16),
+    ("w8a16_multi_tile", 300, 256, 256, 4, 2, 0, moe.AUTO, syn.E4M3, syn.BF16),
 ]
+
+
+def _act(dt, a):
+    return dev_u8(a) if dt == syn.E4M3 else dev_bf16(a)
 
 
 @pytest.mark.parametrize("case", GEMM_CASES, ids=lambda c: c[0])
 def test_grouped_gemm_swiglu_matches_oracle(case):
-    name, T, H, I, E, k, ns, variant, fp8 = case
-    dt = syn.E4M3 if fp8 else syn.BF16
-    wl = syn.Workload(name, T=T, H=H, I=I, E=E, k=k, n_shared=ns, wdtype=dt, adtype=dt, seed=21)
+    name, T, H, I, E, k, ns, variant, wdt, adt = case
+    fp8a = adt == syn.E4M3
+    wl = syn.Workload(name, T=T, H=H, I=I, E=E, k=k, n_shared=ns, wdtype=wdt, adtype=adt, seed=21)
     s = _shape(wl, variant=variant)
     c, o, r, v = _segments(T, E, k, ns, 16, 3)
     mr = moe.max_rows(s)
-    xp = syn.random_rows(1, "xp", mr, H, dt)
+    xp = syn.random_rows(1, "xp", mr, H, adt)
     w13, s13 = syn.expert_weights(wl, "w13")
-    a1 = 1.0 / 64 if fp8 else 1.0
-    a2 = 0.02 if fp8 else 1.0
-    h = torch.zeros((mr, I * (1 if fp8 else 2)), dtype=torch.uint8, device="cuda")
+    a1 = 1.0 / 64 if fp8a else 1.0
+    a2 = 0.02 if fp8a else 1.0
+    h = torch.zeros((mr, I * (1 if fp8a else 2)), dtype=torch.uint8, device="cuda")
     ws = moe.workspace(s)
     moe.reset_device_status(ws)
-    moe.grouped_gemm_swiglu(s, dev_u8(xp) if fp8 else dev_bf16(xp), dev_w(wl, w13),
-                            torch.from_numpy(s13).cuda() if fp8 else None, a1, a2,
+    moe.grouped_gemm_swiglu(s, _act(adt, xp), dev_w(wl, w13),
+                            torch.from_numpy(s13).cuda() if wdt == syn.E4M3 else None, a1, a2,
                             torch.from_numpy(o).cuda(), h, ws)
     torch.cuda.synchronize()
     assert moe.device_status(ws) == 0
     total = o[-1]
-    ref = orc.expert_swiglu(xp[:total], o, w13, dt, s13 if fp8 else None, dt, a1)
+    ref = orc.expert_swiglu(xp[:total], o, w13, wdt, s13 if wdt == syn.E4M3 else None, adt, a1)
     hv = h.cpu().numpy()[:total]
-    if fp8:
+    if fp8a:
         got = orc.e4m3_decode(hv.ravel()).reshape(total, I) * a2
         refq = orc.e4m3_decode(orc.e4m3_encode(ref / a2).ravel()).reshape(total, I) * a2
         assert rel_err(got, refq, "e4m3") <= FP8_TOL
@@ -218,26 +226,27 @@ def test_grouped_gemm_swiglu_matches_oracle(case):
 
 @pytest.mark.parametrize("case", GEMM_CASES, ids=lambda c: c[0])
 def test_grouped_gemm_down_matches_oracle(case):
-    name, T, H, I, E, k, ns, variant, fp8 = case
-    dt = syn.E4M3 if fp8 else syn.BF16
-    wl = syn.Workload(name, T=T, H=H, I=I, E=E, k=k, n_shared=ns, wdtype=dt, adtype=dt, seed=22)
+    name, T, H, I, E, k, ns, variant, wdt, adt = case
+    fp8a = adt == syn.E4M3
+    wl = syn.Workload(name, T=T, H=H, I=I, E=E, k=k, n_shared=ns, wdtype=wdt, adtype=adt, seed=22)
     s = _shape(wl, variant=variant)
     c, o, r, v = _segments(T, E, k, ns, 16, 4)
     mr = moe.max_rows(s)
-    hin = syn.random_rows(2, "h", mr, I, dt, std=0.5)
+    hin = syn.random_rows(2, "h", mr, I, adt, std=0.5)
     w2, s2 = syn.expert_weights(wl, "w2")
-    a2 = 0.01 if fp8 else 1.0
+    a2 = 0.01 if fp8a else 1.0
     y = torch.zeros((mr, H), dtype=torch.float32, device="cuda")
     ws = moe.workspace(s)
     moe.reset_device_status(ws)
-    moe.grouped_gemm_down(s, dev_u8(hin) if fp8 else dev_bf16(hin), dev_w(wl, w2),
-                          torch.from_numpy(s2).cuda() if fp8 else None, a2, torch.from_numpy(o).cuda(), y, ws)
+    moe.grouped_gemm_down(s, _act(adt, hin), dev_w(wl, w2),
+                          torch.from_numpy(s2).cuda() if wdt == syn.E4M3 else None, a2,
+                          torch.from_numpy(o).cuda(), y, ws)
     torch.cuda.synchronize()
     assert moe.device_status(ws) == 0
     total = o[-1]
-    ref = orc.expert_down(hin[:total], o, w2, dt, s2 if fp8 else None, dt, a2)
+    ref = orc.expert_down(hin[:total], o, w2, wdt, s2 if wdt == syn.E4M3 else None, adt, a2)
     got = y.cpu().numpy()[:total].astype(np.float64)
-    assert rel_err(got, ref) <= (1e-4 if not fp8 else 1e-4)
+    assert rel_err(got, ref) <= 1e-4
 
 
 def test_combine_matches_oracle():
@@ -337,3 +346,18 @@ def test_fused_fp8_weights_and_activations(variant):
     got = L.run()
     assert L.status() == 0
     assert rel_err(got, ref, "bf16") <= FP8_TOL
+
+
+@pytest.mark.parametrize("T", [1, 8, 32, 128])
+def test_fused_fp8_weights_bf16_activations_sigmoid_shared(T):
+    """DeepSeek-V3-shaped routing (E=256, top-8 sigmoid x2.5, one shared
+    expert, E4M3 weights, bf16 activations) at reduced H and I."""
+    wl = syn.Workload("dsv3_small", T=T, H=1024, I=256, E=256, k=8, n_shared=1, gate=syn.SIGMOID,
+                      routed_scale=2.5, wdtype=syn.E4M3, seed=8)
+    d = syn.make_inputs(wl)
+    ref = oracle_forward(wl, d)
+    L = Layer(wl, d)
+    got = L.run()
+    assert L.status() == 0
+    assert rel_err(got, ref, "bf16") <= FP8_TOL
+    assert np.array_equal(got, L.run())
