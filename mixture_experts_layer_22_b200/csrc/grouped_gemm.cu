@@ -75,17 +75,19 @@ struct Cfg {
     static constexpr int kStagesW8 = kStagesW8Fit > 10 ? 10 : kStagesW8Fit;
     static constexpr int kStages = kW8 ? kStagesW8 : kStagesFull;
     static constexpr int kDynSmem = (kW8 ? kStagesW8 * kStageW8 : kStagesFull * kStage) + 1024;
-    static constexpr int kThreads = kW8 ? 448 : 192;
+    static constexpr int kThreads = kW8 ? 480 : 192;   // kW8: + 8 converter warps + a 2nd MMA warp
     static constexpr int kAccCols = kSwap ? kBN : 256;      // fp32 columns per accumulator
+    // kW8: each accumulator buffer has two halves (one per MMA warp / K half)
+    static constexpr int kAccSplit = kW8 ? 2 : 1;
     static constexpr int kTmemCols = kW8 ? 512 : ((2 * kAccCols) <= 32 ? 32 : 2 * kAccCols);
-    static constexpr int kAColBase = 2 * kAccCols;                   // first TMEM column of the A slabs
-    static constexpr int kAStages = 8;                               // A slabs of 32 columns
+    static constexpr int kAColBase = 2 * kAccSplit * kAccCols;       // first TMEM column of the A slabs
+    static constexpr int kAStages = 8;                               // A slabs of 32 columns (4 pairs)
     static constexpr int kRowsTile = kSwap ? kBN : 128;     // token rows per tile
     static constexpr int kFeatTile = kMode == 0 ? (kSwap ? 64 : 128) : (kSwap ? 128 : 256);
     static constexpr int kKStage = (kFp8 || kW8) ? 128 : 64;   // K elements per work step
     static constexpr uint32_t kFmt = kFp8 ? 0u : 1u;
     static_assert(kW8 ? kStagesW8 >= 4 : kStagesFull >= 2, "smem ring too small");
-    static_assert(!kW8 || (kSwap && !kFp8 && kBN <= 128), "E4M3-weight/bf16-activation path: Swap-AB, BN <= 128");
+    static_assert(!kW8 || (kSwap && !kFp8 && kBN <= 64), "E4M3-weight/bf16-activation path: Swap-AB, BN <= 64");
     static_assert(!kW8 || kAColBase + kAStages * 32 <= 512, "tensor memory for the A slabs");
     static_assert(kTmemCols <= 512, "tensor memory");
 };
@@ -205,23 +207,37 @@ __device__ __forceinline__ uint32_t e4m3_code(float v)
     return static_cast<uint32_t>(__nv_cvt_float_to_fp8(v, __NV_SATFINITE, __NV_E4M3)) & 0xFFu;
 }
 
+// Four E4M3 codes (one 32-bit word, first code in the low byte) -> four bf16
+// values (two bf16x2 words, K order), exactly.  Each code's bits are placed
+// so that the bf16 exponent field holds the E4M3 exponent field unchanged
+// (s 0000 eeee mmm 0000), which is the bf16 number w * 2^-120 for normal AND
+// subnormal codes; one bf16 multiply by 2^120 then gives w exactly.  Codes
+// 0x7F/0xFF (NaN) are not valid weights.
+__device__ __forceinline__ void e4m3x4_to_bf16(uint32_t w, uint32_t &lo, uint32_t &hi)
+{
+    const uint32_t two120 = 0x7B807B80u;   // bf16x2 {2^120, 2^120}
+    uint32_t t0 = __byte_perm(w, 0u, 0x1404u);   // {b1 << 8, b0 << 8}
+    uint32_t t1 = __byte_perm(w, 0u, 0x3424u);   // {b3 << 8, b2 << 8}
+    t0 >>= 4;                                    // {b1 << 4, b0 << 4}: sign at bit 11
+    t1 >>= 4;
+    t0 += 15u * (t0 & 0x08000800u);              // move the sign from bit 11 to bit 15
+    t1 += 15u * (t1 & 0x08000800u);
+    asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(lo) : "r"(t0), "r"(two120));
+    asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(hi) : "r"(t1), "r"(two120));
+}
+
 // 64 E4M3 codes (four 16-byte chunks of one swizzled 128-byte row) -> 64
-// bf16 values packed two per 32-bit word, K order.  Exact: every E4M3 value
-// is an fp16 value and a bf16 value.
+// bf16 values packed two per 32-bit word, K order.
 __device__ __forceinline__ void e4m3x64_to_bf16(const uint8_t *row, int r, int half, uint32_t (&o)[32])
 {
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
         const int c = 4 * half + q;
         const uint4 v = *reinterpret_cast<const uint4 *>(row + ((c ^ (r & 7)) << 4));
-        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const uint16_t pair = static_cast<uint16_t>(w[i >> 1] >> ((i & 1) * 16));
-            const uint32_t h2 = cvt_e4m3x2_f16x2(pair);
-            const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&h2));
-            o[q * 8 + i] = pack_bf16x2(f.x, f.y);
-        }
+        e4m3x4_to_bf16(v.x, o[q * 8 + 0], o[q * 8 + 1]);
+        e4m3x4_to_bf16(v.y, o[q * 8 + 2], o[q * 8 + 3]);
+        e4m3x4_to_bf16(v.z, o[q * 8 + 4], o[q * 8 + 5]);
+        e4m3x4_to_bf16(v.w, o[q * 8 + 6], o[q * 8 + 7]);
     }
 }
 
@@ -248,7 +264,7 @@ __global__ void __launch_bounds__(Cfg<kMode, kSwap, kFp8, kBN, kW8>::kThreads, 1
     __shared__ int s_off[kMaxExpertsTotal + 1];
     __shared__ int s_prefix[kMaxExpertsTotal + 1];
     __shared__ __align__(8) uint64_t s_full[C::kStages], s_empty[C::kStages];
-    __shared__ __align__(8) uint64_t s_tfull[2], s_tempty[2], s_drain;
+    __shared__ __align__(8) uint64_t s_tfull[2], s_tempty[2], s_drain, s_drain2;
     __shared__ uint32_t s_tmem_base;
     __shared__ volatile int s_abort;
     __shared__ int s_is_last;
@@ -266,19 +282,20 @@ __global__ void __launch_bounds__(Cfg<kMode, kSwap, kFp8, kBN, kW8>::kThreads, 1
         s_abort = 0;
         for (int i = 0; i < C::kStages; ++i) {
             mbar_init(smem_u32(&s_full[i]), 1);
-            // kW8: the stage is free once the 8 converter warps have read the
-            // raw tile and the MMA has read the activations (one commit)
-            mbar_init(smem_u32(&s_empty[i]), kW8 ? 9 : 1);
+            // kW8: the stage is free once its 4 converter warps have read the
+            // raw tile and both MMA warps have read the activations
+            mbar_init(smem_u32(&s_empty[i]), kW8 ? 6 : 1);
         }
         for (int i = 0; i < 2; ++i) {
-            mbar_init(smem_u32(&s_tfull[i]), 1);
+            mbar_init(smem_u32(&s_tfull[i]), kW8 ? 2 : 1);
             mbar_init(smem_u32(&s_tempty[i]), 4);
         }
         mbar_init(smem_u32(&s_drain), 1);
+        mbar_init(smem_u32(&s_drain2), 1);
         if (kW8) {
-            for (int i = 0; i < kAN; ++i) {
-                mbar_init(smem_u32(&s_a_full[i]), 4);         // the four warps of one K half
-                mbar_init(smem_u32(&s_a_empty[i]), 1);
+            for (int i = 0; i < kAN; ++i) {                    // one barrier pair per slab pair
+                mbar_init(smem_u32(&s_a_full[i]), 4);         // the four warps of a converter group
+                mbar_init(smem_u32(&s_a_empty[i]), 2);        // both MMA warps
             }
         }
         fence_mbar_init();
@@ -380,12 +397,14 @@ __global__ void __launch_bounds__(Cfg<kMode, kSwap, kFp8, kBN, kW8>::kThreads, 1
             }
             if (!ok) drain_ring(s_full, C::kStages, stage, phase, in_flight);
         }
-    } else if (kW8 && warp >= 6) {
+    } else if (kW8 && warp >= 6 && warp <= 13) {
         // ================= E4M3 -> bf16 converters (warps 6..13) ============
-        // Warp w converts K half (w - 6) / 4 of each stage for the 32 weight
-        // rows of its tensor-memory lane quarter (w % 4): thread = one row,
-        // 64 codes -> 32 packed columns, stored into an A slab with tcgen05.st.
-        const int half = (warp - 6) >> 2;
+        // Two groups of four warps take alternate stages (group g: stages
+        // j = g, g+2, ...), so two stages are converted at once.  Warp w
+        // covers the 32 weight rows of its tensor-memory lane quarter (w % 4):
+        // thread = one row, both K halves (2 x 64 codes -> 2 x 32 packed
+        // columns), stored into slab pair j % 4 with tcgen05.st.
+        const int group = (warp - 6) >> 2;
         const int q = warp & 3;
         const int r = q * 32 + lane;
         const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
@@ -397,25 +416,28 @@ __global__ void __launch_bounds__(Cfg<kMode, kSwap, kFp8, kBN, kW8>::kThreads, 1
         bool ok = true;
         while (ok && iter_next<C::kRowsTile>(I, S, s_prefix, s_off, Et, n_ft, it)) {
             for (int kk = it.kb; kk < it.ke; ++kk, ++j) {
-                // half-step 2j + half uses slab (2j + half) % kAStages
-                const int qs = 2 * j + half;
-                const int as = qs % C::kAStages;
-                const uint32_t aph = static_cast<uint32_t>(qs / C::kAStages) & 1u;
-                if (!mbar_wait(smem_u32(&s_full[stage]), phase, &s_abort) ||
-                    !mbar_wait(smem_u32(&s_a_empty[as]), aph ^ 1u, &s_abort)) {
-                    ok = false;
-                    break;
-                }
-                tc_fence_after();
-                uint32_t o[32];
-                e4m3x64_to_bf16(tiles + stage * C::kStageW8 + r * 128, r, half, o);
-                tmem_st32(tmem_base + lane_base + C::kAColBase + as * 32, o);
-                tmem_wait_st();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) {
-                    mbar_arrive(smem_u32(&s_a_full[as]));
-                    mbar_arrive(smem_u32(&s_empty[stage]));
+                if ((j & 1) == group) {
+                    const int pr = j & 3;
+                    const uint32_t aph = static_cast<uint32_t>(j >> 2) & 1u;
+                    if (!mbar_wait(smem_u32(&s_full[stage]), phase, &s_abort) ||
+                        !mbar_wait(smem_u32(&s_a_empty[pr]), aph ^ 1u, &s_abort)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint8_t *row = tiles + stage * C::kStageW8 + r * 128;
+                    uint32_t o[32];
+                    e4m3x64_to_bf16(row, r, 0, o);
+                    tmem_st32(tmem_base + lane_base + C::kAColBase + (2 * pr) * 32, o);
+                    e4m3x64_to_bf16(row, r, 1, o);
+                    tmem_st32(tmem_base + lane_base + C::kAColBase + (2 * pr + 1) * 32, o);
+                    tmem_wait_st();
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) {
+                        mbar_arrive(smem_u32(&s_a_full[pr]));
+                        mbar_arrive(smem_u32(&s_empty[stage]));
+                    }
                 }
                 if (++stage == C::kStages) {
                     stage = 0;
@@ -423,10 +445,14 @@ __global__ void __launch_bounds__(Cfg<kMode, kSwap, kFp8, kBN, kW8>::kThreads, 1
                 }
             }
         }
-    } else if (kW8 && warp == 1) {
-        // ================= MMA issuer (A = bf16 slabs in TMEM, B = smem) ====
+    } else if (kW8 && (warp == 1 || warp == 14)) {
+        // ================= MMA issuers (A = bf16 slabs in TMEM, B = smem) ===
+        // Warp 1 issues the K half 0 MMAs of every stage, warp 14 those of
+        // K half 1, each into its own half of the accumulator buffer; the
+        // epilogue adds the two halves.
         if (lane == 0) {
-            int stage = 0, acc = 0, qs = 0;
+            const int hh = warp == 1 ? 0 : 1;
+            int stage = 0, acc = 0, j = 0;
             uint32_t phase = 0, acc_phase = 0;
             ItemIter I;
             iter_init(I, S, blockIdx.x);
@@ -435,33 +461,28 @@ __global__ void __launch_bounds__(Cfg<kMode, kSwap, kFp8, kBN, kW8>::kThreads, 1
             while (ok && iter_next<C::kRowsTile>(I, S, s_prefix, s_off, Et, n_ft, it)) {
                 if (!mbar_wait(smem_u32(&s_tempty[acc]), acc_phase ^ 1u, &s_abort)) break;
                 tc_fence_after();
-                const uint32_t d = tmem_base + acc * C::kAccCols;
+                const uint32_t d = tmem_base + (acc * 2 + hh) * C::kAccCols;
                 const int seg = s_off[it.e + 1] - s_off[it.e];
                 const int n = min(C::kRowsTile, seg - it.rt * C::kRowsTile);
                 const uint32_t idesc = idesc_make(1u, 128, n);
-                for (int kk = it.kb; ok && kk < it.ke; ++kk) {
-                    if (!mbar_wait(smem_u32(&s_full[stage]), phase, &s_abort)) {
+                for (int kk = it.kb; kk < it.ke; ++kk, ++j) {
+                    const int pr = j & 3;
+                    // the activation rows landed with the stage (full); the
+                    // converted weight slabs with the pair's a_full
+                    if (!mbar_wait(smem_u32(&s_full[stage]), phase, &s_abort) ||
+                        !mbar_wait(smem_u32(&s_a_full[pr]), static_cast<uint32_t>(j >> 2) & 1u, &s_abort)) {
                         ok = false;
                         break;
                     }
-                    for (int hh = 0; hh < 2; ++hh, ++qs) {
-                        const int as = qs % C::kAStages;
-                        const uint32_t aph = static_cast<uint32_t>(qs / C::kAStages) & 1u;
-                        if (!mbar_wait(smem_u32(&s_a_full[as]), aph, &s_abort)) {
-                            ok = false;
-                            break;
-                        }
-                        tc_fence_after();
-                        const uint32_t ta = tmem_base + C::kAColBase + as * 32;
-                        const uint32_t sb = smem_u32(tiles + stage * C::kStageW8 + C::kStageA + hh * C::kStageB);
+                    tc_fence_after();
+                    const uint32_t ta = tmem_base + C::kAColBase + (2 * pr + hh) * 32;
+                    const uint32_t sb = smem_u32(tiles + stage * C::kStageW8 + C::kStageA + hh * C::kStageB);
+                    const uint64_t bd0 = sdesc_k_sw128(sb);
 #pragma unroll
-                        for (int s4 = 0; s4 < 4; ++s4) {
-                            const uint32_t accum = (kk > it.kb || hh > 0 || s4 > 0) ? 1u : 0u;
-                            mma_bf16_tmem_a(d, ta + s4 * 8, sdesc_k_sw128(sb + s4 * 32), idesc, accum);
-                        }
-                        mma_commit(smem_u32(&s_a_empty[as]));
-                    }
-                    if (!ok) break;
+                    for (int s4 = 0; s4 < 4; ++s4)
+                        mma_bf16_tmem_a(d, ta + s4 * 8, bd0 + static_cast<uint64_t>(s4 * 2), idesc,
+                                        (kk > it.kb || s4 > 0) ? 1u : 0u);
+                    mma_commit(smem_u32(&s_a_empty[pr]));
                     mma_commit(smem_u32(&s_empty[stage]));
                     if (++stage == C::kStages) {
                         stage = 0;
@@ -475,9 +496,10 @@ __global__ void __launch_bounds__(Cfg<kMode, kSwap, kFp8, kBN, kW8>::kThreads, 1
                     acc_phase ^= 1u;
                 }
             }
-            mma_commit(smem_u32(&s_drain));
+            uint64_t *dr = warp == 1 ? &s_drain : &s_drain2;
+            mma_commit(smem_u32(dr));
             volatile int no_abort = 0;
-            mbar_wait(smem_u32(&s_drain), 0, &no_abort);
+            mbar_wait(smem_u32(dr), 0, &no_abort);
         }
     } else if (!kW8 && warp == 0) {
         // ================= TMA producer =================
@@ -606,7 +628,18 @@ __global__ void __launch_bounds__(Cfg<kMode, kSwap, kFp8, kBN, kW8>::kThreads, 1
             const int row0 = s_off[it.e] + it.rt * C::kRowsTile;
             const int rows = min(C::kRowsTile, seg - it.rt * C::kRowsTile);
             const float sc = p.ascale * (p.wscale ? __ldg(&p.wscale[it.e]) : 1.0f);
-            const uint32_t tacc = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * C::kAccCols;
+            const uint32_t tacc = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * C::kAccSplit * C::kAccCols;
+            // 16 accumulator columns starting at c0 (kW8: sum of the two halves)
+            auto ld_acc16 = [&](int c0, uint32_t (&v)[16]) {
+                tmem_ld16(tacc + c0, v);
+                if constexpr (kW8) {
+                    uint32_t w2[16];
+                    tmem_ld16(tacc + C::kAccCols + c0, w2);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int i2 = 0; i2 < 16; ++i2) v[i2] = __float_as_uint(__uint_as_float(v[i2]) + __uint_as_float(w2[i2]));
+                }
+            };
             const int ncols = kSwap ? rows : 256;
             if (!it.partial) {
                 if (kSwap && kMode == 0) {
@@ -614,7 +647,7 @@ __global__ void __launch_bounds__(Cfg<kMode, kSwap, kFp8, kBN, kW8>::kThreads, 1
                     const int f0 = it.ft * 64;
                     for (int c0 = 0; c0 < ncols; c0 += 16) {
                         uint32_t v[16];
-                        tmem_ld16(tacc + c0, v);
+                        ld_acc16(c0, v);
                         tmem_wait_ld();
                         if (q >= 2)
 #pragma unroll
@@ -639,7 +672,7 @@ __global__ void __launch_bounds__(Cfg<kMode, kSwap, kFp8, kBN, kW8>::kThreads, 1
                     const int h0 = it.ft * 128;
                     for (int c0 = 0; c0 < ncols; c0 += 16) {
                         uint32_t v[16];
-                        tmem_ld16(tacc + c0, v);
+                        ld_acc16(c0, v);
                         tmem_wait_ld();
 #pragma unroll
                         for (int j = 0; j < 16; ++j)
@@ -685,7 +718,7 @@ __global__ void __launch_bounds__(Cfg<kMode, kSwap, kFp8, kBN, kW8>::kThreads, 1
                     for (int c0 = 0; c0 < 256; c0 += 16) {
                         if (h0 + c0 >= p.n_feat) break;
                         uint32_t v[16];
-                        tmem_ld16(tacc + c0, v);
+                        ld_acc16(c0, v);
                         tmem_wait_ld();
                         if (valid) {
                             float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(p.out) +
@@ -705,7 +738,7 @@ __global__ void __launch_bounds__(Cfg<kMode, kSwap, kFp8, kBN, kW8>::kThreads, 1
                 float *slot = p.partials + static_cast<size_t>(it.slot) * 128 * C::kAccCols;
                 for (int c0 = 0; c0 < ncols; c0 += 16) {
                     uint32_t v[16];
-                    tmem_ld16(tacc + c0, v);
+                    ld_acc16(c0, v);
                     tmem_wait_ld();
 #pragma unroll
                     for (int j = 0; j < 16; ++j) __stcg(&slot[(c0 + j) * 128 + r], __uint_as_float(v[j]));
@@ -909,8 +942,7 @@ cudaError_t launch_grouped_gemm(const moe_shape_t &s, const GemmPlan &p, const G
     switch (p.bn) {                          \
     case 16: MOE_W8(MODE, 16); break;        \
     case 32: MOE_W8(MODE, 32); break;        \
-    case 64: MOE_W8(MODE, 64); break;        \
-    default: MOE_W8(MODE, 128); break;       \
+    default: MOE_W8(MODE, 64); break;        \
     }
         if (a.mode == 0) { MOE_W8_BY_BN(0) } else { MOE_W8_BY_BN(1) }
 #undef MOE_W8_BY_BN

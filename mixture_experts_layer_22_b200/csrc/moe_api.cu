@@ -46,9 +46,9 @@ GemmPlan plan_gemm(const moe_shape_t &s)
     if (p.swap) {
         const int rows = (s.T + s.pad - 1) / s.pad * s.pad;   // worst case rows of one expert
         int bn = 16;
-        // the E4M3-weight path keeps converted weight slabs in tensor memory
-        // next to the accumulators, which caps its token tile at 128 rows
-        const int cap = (s.wdtype == MOE_E4M3 && s.adtype == MOE_BF16) ? 128 : 256;
+        // the E4M3-weight path keeps converted weight slabs and split
+        // accumulators in tensor memory, which caps its token tile at 64 rows
+        const int cap = (s.wdtype == MOE_E4M3 && s.adtype == MOE_BF16) ? 64 : 256;
         while (bn < rows && bn < cap) bn <<= 1;
         p.bn = bn;
     } else {

@@ -361,3 +361,44 @@ def test_fused_fp8_weights_bf16_activations_sigmoid_shared(T):
     assert L.status() == 0
     assert rel_err(got, ref, "bf16") <= FP8_TOL
     assert np.array_equal(got, L.run())
+
+
+@pytest.mark.parametrize("mode", ["swiglu", "down"])
+def test_e4m3_weight_expansion_is_exact(mode):
+    """E4M3 weights drawn from every finite code (subnormals included), scale
+    1: the E4M3-weight GEMM must equal the bf16-weight GEMM on the identical
+    bf16 values up to fp32 summation order, which checks that the kernel's
+    E4M3 -> bf16 expansion is exact."""
+    T, H, I, E, k = 32, 512, 256, 4, 2
+    rng = np.random.default_rng(12)
+    codes = np.array([c for c in range(256) if c not in (0x7F, 0xFF)], dtype=np.uint8)
+    rows_w = 2 * I if mode == "swiglu" else H
+    cols_w = H if mode == "swiglu" else I
+    q = rng.choice(codes, size=(E, rows_w, cols_w)).astype(np.uint8)
+    wbits = orc.bf16_encode(orc.e4m3_decode(q.ravel())).reshape(q.shape)
+    ones = torch.ones(E, dtype=torch.float32, device="cuda")
+    c, o, r, v = _segments(T, E, k, 0, 16, 5)
+    wl8 = syn.Workload("w8", T=T, H=H, I=I, E=E, k=k, wdtype=syn.E4M3)
+    wl16 = syn.Workload("w16", T=T, H=H, I=I, E=E, k=k)
+    s8, s16 = _shape(wl8), _shape(wl16, variant=moe.SWAP_AB)
+    mr = moe.max_rows(s16)
+    offs = torch.from_numpy(o).cuda()
+    cols_a = H if mode == "swiglu" else I
+    act = dev_bf16(syn.random_rows(6, "a", mr, cols_a, syn.BF16, std=0.05))
+    outs = []
+    for s, w, sc in ((s8, dev_u8(q), ones), (s16, dev_bf16(wbits), None)):
+        ws = moe.workspace(s)
+        moe.reset_device_status(ws)
+        if mode == "swiglu":
+            out = torch.zeros((mr, I), dtype=torch.bfloat16, device="cuda")
+            moe.grouped_gemm_swiglu(s, act, w, sc, 1.0, 1.0, offs, out, ws)
+        else:
+            out = torch.zeros((mr, H), dtype=torch.float32, device="cuda")
+            moe.grouped_gemm_down(s, act, w, sc, 1.0, offs, out, ws)
+        torch.cuda.synchronize()
+        assert moe.device_status(ws) == 0
+        outs.append(out.float().cpu().numpy()[:o[-1]].astype(np.float64))
+    if mode == "swiglu":
+        assert rel_err(outs[0], outs[1], "bf16") <= 1e-3
+    else:
+        assert rel_err(outs[0], outs[1]) <= 1e-5
