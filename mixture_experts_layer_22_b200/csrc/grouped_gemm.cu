@@ -60,8 +60,13 @@ struct GemmParams {
 
 template <int kMode, bool kSwap, bool kFp8, int kBN, bool kW8 = false>
 struct Cfg {
-    static constexpr int kStageA = 128 * 128;               // 128 rows x 128 bytes
-    static constexpr int kStageB = kBN * 128;
+    // K bytes per operand row and stage (128: the 128-byte swizzle; 64-byte
+    // rows with the 64-byte swizzle are supported by the loads and
+    // descriptors but measured slower for the normal order on B200).
+    static constexpr int kRowBytes = 128;
+    static constexpr int kMmaPerStage = kRowBytes / 32;     // 32 bytes of K per MMA
+    static constexpr int kStageA = 128 * kRowBytes;          // 128 rows
+    static constexpr int kStageB = kBN * kRowBytes;
     static constexpr int kStage = kStageA + kStageB;
     static constexpr int kDynBudget = 205 * 1024;
     static constexpr int kStagesRaw = kDynBudget / kStage;
@@ -75,7 +80,11 @@ struct Cfg {
     static constexpr int kStagesW8 = kStagesW8Fit > 10 ? 10 : kStagesW8Fit;
     static constexpr int kStages = kW8 ? kStagesW8 : kStagesFull;
     static constexpr int kDynSmem = (kW8 ? kStagesW8 * kStageW8 : kStagesFull * kStage) + 1024;
-    static constexpr int kThreads = kW8 ? 480 : 192;   // kW8: + 8 converter warps + a 2nd MMA warp
+    // epilogue warps 2 .. 2+kEpiWarps-1; the normal order uses two per
+    // tensor-memory lane quarter, each taking half of the tile's columns
+    static constexpr int kEpiWarps = kSwap ? 4 : 8;
+    static constexpr int kEpiThreads = 32 * kEpiWarps;
+    static constexpr int kThreads = kW8 ? 480 : 64 + kEpiThreads;   // kW8: + 8 converters + a 2nd MMA warp
     static constexpr int kAccCols = kSwap ? kBN : 256;      // fp32 columns per accumulator
     // kW8: each accumulator buffer has two halves (one per MMA warp / K half)
     static constexpr int kAccSplit = kW8 ? 2 : 1;
@@ -84,7 +93,7 @@ struct Cfg {
     static constexpr int kAStages = 8;                               // A slabs of 32 columns (4 pairs)
     static constexpr int kRowsTile = kSwap ? kBN : 128;     // token rows per tile
     static constexpr int kFeatTile = kMode == 0 ? (kSwap ? 64 : 128) : (kSwap ? 128 : 256);
-    static constexpr int kKStage = (kFp8 || kW8) ? 128 : 64;   // K elements per work step
+    static constexpr int kKStage = (kFp8 || kW8) ? kRowBytes : kRowBytes / 2;   // K elements per work step
     static constexpr uint32_t kFmt = kFp8 ? 0u : 1u;
     static_assert(kW8 ? kStagesW8 >= 4 : kStagesFull >= 2, "smem ring too small");
     static_assert(!kW8 || (kSwap && !kFp8 && kBN <= 64), "E4M3-weight/bf16-activation path: Swap-AB, BN <= 64");
@@ -191,9 +200,12 @@ __device__ __forceinline__ bool iter_next(ItemIter &I, const Sched &S, const int
     return true;
 }
 
+// SiLU(g) * u with the hardware exponential and an approximate reciprocal
+// (a few ulp of fp32: far below the bf16 / E4M3 rounding of h).  For very
+// negative g, 1 + e^-g overflows to +inf and the quotient is -0.
 __device__ __forceinline__ float silu_mul(float g, float u)
 {
-    return g / (1.0f + __expf(-g)) * u;
+    return __fdividef(g, 1.0f + __expf(-g)) * u;
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b)
@@ -288,7 +300,7 @@ __global__ void __launch_bounds__(Cfg<kMode, kSwap, kFp8, kBN, kW8>::kThreads, 1
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(smem_u32(&s_tfull[i]), kW8 ? 2 : 1);
-            mbar_init(smem_u32(&s_tempty[i]), 4);
+            mbar_init(smem_u32(&s_tempty[i]), C::kEpiWarps);
         }
         mbar_init(smem_u32(&s_drain), 1);
         mbar_init(smem_u32(&s_drain2), 1);
@@ -504,7 +516,11 @@ __global__ void __launch_bounds__(Cfg<kMode, kSwap, kFp8, kBN, kW8>::kThreads, 1
     } else if (!kW8 && warp == 0) {
         // ================= TMA producer =================
         if (lane == 0) {
-            const uint64_t pol_w = policy_evict_first();
+            // Swap-AB (few token rows per expert) streams every weight byte
+            // once: keep it from displacing the reused activations.  In the
+            // normal order a weight tile is reused by all of the expert's row
+            // tiles, so it gets the default policy.
+            const uint64_t pol_w = kSwap ? policy_evict_first() : policy_evict_normal();
             const uint64_t pol_x = policy_evict_last();
             int stage = 0;
             uint32_t phase = 0;
@@ -524,24 +540,24 @@ __global__ void __launch_bounds__(Cfg<kMode, kSwap, kFp8, kBN, kW8>::kThreads, 1
                     }
                     const uint32_t fb = smem_u32(&s_full[stage]);
                     // Swap-AB: only the tile's own token rows (16-row boxes)
-                    mbar_arrive_expect_tx(fb, kSwap ? C::kStageA + rows * 128 : C::kStage);
+                    mbar_arrive_expect_tx(fb, kSwap ? C::kStageA + rows * C::kRowBytes : C::kStage);
                     const uint32_t sa = smem_u32(tiles + stage * C::kStage);
                     const uint32_t sb = sa + C::kStageA;
                     const int kx = kk * C::kKStage;
                     if (kSwap) {
                         if (kMode == 0) {
                             tma_load_2d(sa, &tm_w, fb, kx, wbase + it.ft * 64, pol_w);
-                            tma_load_2d(sa + 64 * 128, &tm_w, fb, kx, wbase + p.n_feat + it.ft * 64, pol_w);
+                            tma_load_2d(sa + 64 * C::kRowBytes, &tm_w, fb, kx, wbase + p.n_feat + it.ft * 64, pol_w);
                         } else {
                             tma_load_2d(sa, &tm_w, fb, kx, wbase + it.ft * 128, pol_w);
                         }
                         for (int rr = 0; rr < rows; rr += 16)
-                            tma_load_2d(sb + rr * 128, &tm_x, fb, kx, row0 + rr, pol_x);
+                            tma_load_2d(sb + rr * C::kRowBytes, &tm_x, fb, kx, row0 + rr, pol_x);
                     } else {
                         tma_load_2d(sa, &tm_x, fb, kx, row0, pol_x);
                         if (kMode == 0) {
                             tma_load_2d(sb, &tm_w, fb, kx, wbase + it.ft * 128, pol_w);
-                            tma_load_2d(sb + 128 * 128, &tm_w, fb, kx, wbase + p.n_feat + it.ft * 128, pol_w);
+                            tma_load_2d(sb + 128 * C::kRowBytes, &tm_w, fb, kx, wbase + p.n_feat + it.ft * 128, pol_w);
                         } else {
                             tma_load_2d(sb, &tm_w, fb, kx, wbase + it.ft * 256, pol_w);
                         }
@@ -585,9 +601,9 @@ __global__ void __launch_bounds__(Cfg<kMode, kSwap, kFp8, kBN, kW8>::kThreads, 1
                     const uint32_t sa = smem_u32(tiles + stage * C::kStage);
                     const uint32_t sb = sa + C::kStageA;
 #pragma unroll
-                    for (int s = 0; s < 4; ++s) {
-                        const uint64_t ad = sdesc_k_sw128(sa + s * 32);
-                        const uint64_t bd = sdesc_k_sw128(sb + s * 32);
+                    for (int s = 0; s < C::kMmaPerStage; ++s) {
+                        const uint64_t ad = C::kRowBytes == 128 ? sdesc_k_sw128(sa + s * 32) : sdesc_k_sw64(sa + s * 32);
+                        const uint64_t bd = C::kRowBytes == 128 ? sdesc_k_sw128(sb + s * 32) : sdesc_k_sw64(sb + s * 32);
                         const uint32_t accum = (kk > it.kb || s > 0) ? 1u : 0u;
                         if (kFp8) mma_e4m3(d, ad, bd, idesc, accum);
                         else mma_bf16(d, ad, bd, idesc, accum);
@@ -610,11 +626,13 @@ __global__ void __launch_bounds__(Cfg<kMode, kSwap, kFp8, kBN, kW8>::kThreads, 1
             volatile int no_abort = 0;
             mbar_wait(smem_u32(&s_drain), 0, &no_abort);
         }
-    } else if (warp >= 2 && warp <= 5) {
-        // ================= epilogue (warps 2..5) =================
+    } else if (warp >= 2 && warp < 2 + C::kEpiWarps) {
+        // ================= epilogue (warps 2 .. 2+kEpiWarps-1) ==============
         const int q = warp & 3;                 // tensor-memory lane quarter
         const int r = q * 32 + lane;            // accumulator row of this thread
-        const int etid = threadIdx.x - 64;      // 0..127
+        const int etid = threadIdx.x - 64;      // 0 .. kEpiThreads-1
+        const int ch = (warp - 2) >> 2;         // column half (normal order, 8 warps)
+        constexpr int kNch = C::kEpiWarps / 4;  // column halves
         int acc = 0;
         uint32_t acc_phase = 0;
         ItemIter I;
@@ -622,7 +640,7 @@ __global__ void __launch_bounds__(Cfg<kMode, kSwap, kFp8, kBN, kW8>::kThreads, 1
         Item it;
         while (iter_next<C::kRowsTile>(I, S, s_prefix, s_off, Et, n_ft, it)) {
             const bool got = mbar_wait(smem_u32(&s_tfull[acc]), acc_phase, &s_abort);
-            if (!named_bar_and(1, 128, got)) break;   // all four warps agree
+            if (!named_bar_and(1, C::kEpiThreads, got)) break;   // all epilogue warps agree
             tc_fence_after();
             const int seg = s_off[it.e + 1] - s_off[it.e];
             const int row0 = s_off[it.e] + it.rt * C::kRowsTile;
@@ -682,7 +700,7 @@ __global__ void __launch_bounds__(Cfg<kMode, kSwap, kFp8, kBN, kW8>::kThreads, 1
                 } else if (kMode == 0) {
                     const int f0 = it.ft * 128;
                     const bool valid = r < rows;
-                    for (int c0 = 0; c0 < 128; c0 += 16) {
+                    for (int c0 = ch * (128 / kNch); c0 < (ch + 1) * (128 / kNch); c0 += 16) {
                         uint32_t g[16], u[16];
                         tmem_ld16(tacc + c0, g);
                         tmem_ld16(tacc + 128 + c0, u);
@@ -715,7 +733,7 @@ __global__ void __launch_bounds__(Cfg<kMode, kSwap, kFp8, kBN, kW8>::kThreads, 1
                 } else {
                     const int h0 = it.ft * 256;
                     const bool valid = r < rows;
-                    for (int c0 = 0; c0 < 256; c0 += 16) {
+                    for (int c0 = ch * (256 / kNch); c0 < (ch + 1) * (256 / kNch); c0 += 16) {
                         if (h0 + c0 >= p.n_feat) break;
                         uint32_t v[16];
                         ld_acc16(c0, v);
@@ -736,7 +754,7 @@ __global__ void __launch_bounds__(Cfg<kMode, kSwap, kFp8, kBN, kW8>::kThreads, 1
             } else {
                 // ---- one share of a split tile: store the raw partial ----
                 float *slot = p.partials + static_cast<size_t>(it.slot) * 128 * C::kAccCols;
-                for (int c0 = 0; c0 < ncols; c0 += 16) {
+                for (int c0 = ch * (ncols / kNch); c0 < (ch + 1) * (ncols / kNch); c0 += 16) {
                     uint32_t v[16];
                     ld_acc16(c0, v);
                     tmem_wait_ld();
@@ -747,7 +765,7 @@ __global__ void __launch_bounds__(Cfg<kMode, kSwap, kFp8, kBN, kW8>::kThreads, 1
                 __syncwarp();
                 if (lane == 0) mbar_arrive(smem_u32(&s_tempty[acc]));
                 __threadfence();
-                named_bar_sync(1, 128);
+                named_bar_sync(1, C::kEpiThreads);
                 // contributing CTAs of this tile, in K order
                 const long long t_it0 = static_cast<long long>(it.sk_tile) * S.KT;
                 const int c_first = sk_cta_of(t_it0, S);
@@ -756,7 +774,7 @@ __global__ void __launch_bounds__(Cfg<kMode, kSwap, kFp8, kBN, kW8>::kThreads, 1
                     const int old = atomicAdd(&p.counters[it.sk_tile], 1);
                     s_is_last = (old == c_last - c_first);
                 }
-                named_bar_sync(1, 128);
+                named_bar_sync(1, C::kEpiThreads);
                 if (s_is_last) {
                     __threadfence();
                     auto slot_of = [&](int c) -> const float * {
@@ -788,30 +806,32 @@ __global__ void __launch_bounds__(Cfg<kMode, kSwap, kFp8, kBN, kW8>::kThreads, 1
                         }
                     } else if (kMode == 0) {
                         const int f0 = it.ft * 128;
-                        if (etid < rows)
-                            for (int j = 0; j < 128; ++j) {
+                        const int rr = etid & 127, hf = etid >> 7;
+                        if (rr < rows)
+                            for (int j = hf * (128 / kNch); j < (hf + 1) * (128 / kNch); ++j) {
                                 float g = 0.f, u = 0.f;
                                 for (int c = c_first; c <= c_last; ++c) {
                                     const float *ps = slot_of(c);
-                                    g += __ldcg(&ps[j * 128 + etid]);
-                                    u += __ldcg(&ps[(128 + j) * 128 + etid]);
+                                    g += __ldcg(&ps[j * 128 + rr]);
+                                    u += __ldcg(&ps[(128 + j) * 128 + rr]);
                                 }
                                 const float hv = silu_mul(g * sc, u * sc);
-                                const size_t o = static_cast<size_t>(row0 + etid) * p.out_ld + f0 + j;
+                                const size_t o = static_cast<size_t>(row0 + rr) * p.out_ld + f0 + j;
                                 if (kFp8) static_cast<uint8_t *>(p.out)[o] = static_cast<uint8_t>(e4m3_code(hv / p.qscale));
                                 else static_cast<__nv_bfloat16 *>(p.out)[o] = __float2bfloat16_rn(hv);
                             }
                     } else {
                         const int h0 = it.ft * 256;
-                        if (etid < rows)
-                            for (int j = 0; j < 256 && h0 + j < p.n_feat; ++j) {
+                        const int rr = etid & 127, hf = etid >> 7;
+                        if (rr < rows)
+                            for (int j = hf * (256 / kNch); j < (hf + 1) * (256 / kNch) && h0 + j < p.n_feat; ++j) {
                                 float a = 0.f;
-                                for (int c = c_first; c <= c_last; ++c) a += __ldcg(&slot_of(c)[j * 128 + etid]);
-                                static_cast<float *>(p.out)[static_cast<size_t>(row0 + etid) * p.out_ld + h0 + j] = a * sc;
+                                for (int c = c_first; c <= c_last; ++c) a += __ldcg(&slot_of(c)[j * 128 + rr]);
+                                static_cast<float *>(p.out)[static_cast<size_t>(row0 + rr) * p.out_ld + h0 + j] = a * sc;
                             }
                     }
                 }
-                named_bar_sync(1, 128);
+                named_bar_sync(1, C::kEpiThreads);
             }
             if (++acc == 2) {
                 acc = 0;
@@ -853,18 +873,19 @@ static EncodeTiledFn get_encode_fn()
 // 2-D map over a row-major [rows, cols] matrix with 128-byte rows per box
 // and the 128-byte swizzle; box = box_rows x (128 bytes).
 static bool make_map(CUtensorMap *m, const void *base, bool u8, uint64_t rows, uint64_t cols,
-                     uint32_t box_rows)
+                     uint32_t box_rows, uint32_t row_bytes = 128)
 {
     EncodeTiledFn fn = get_encode_fn();
     if (!fn) return false;
     const uint32_t esz = u8 ? 1 : 2;
     cuuint64_t dims[2] = {cols, rows};
     cuuint64_t strides[1] = {cols * esz};
-    cuuint32_t box[2] = {128 / esz, box_rows};
+    cuuint32_t box[2] = {row_bytes / esz, box_rows};
     cuuint32_t estr[2] = {1, 1};
     CUresult r = fn(m, u8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
                     const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                    CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    row_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
@@ -901,8 +922,8 @@ static cudaError_t run_gemm(const moe_shape_t &s, const GemmArgs &a, cudaStream_
     const uint32_t wbox = kSwap ? (kMode == 0 ? 64 : 128) : (kMode == 0 ? 128 : 256);
     const uint32_t xbox = kSwap ? 16 : 128;     // Swap-AB loads token rows in 16-row boxes
     CUtensorMap tm_w, tm_x;
-    if (!make_map(&tm_w, a.wgt, u8w, Et * w_rows, K, wbox) ||
-        !make_map(&tm_x, a.act, u8, a.max_rows, K, xbox)) {
+    if (!make_map(&tm_w, a.wgt, u8w, Et * w_rows, K, wbox, Cf::kRowBytes) ||
+        !make_map(&tm_x, a.act, u8, a.max_rows, K, xbox, Cf::kRowBytes)) {
         *host_err = MOE_ERR_CUDA;
         return cudaSuccess;
     }

@@ -85,6 +85,13 @@ __device__ __forceinline__ uint64_t policy_evict_first()
     return p;
 }
 
+__device__ __forceinline__ uint64_t policy_evict_normal()
+{
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_normal.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+
 __device__ __forceinline__ uint64_t policy_evict_last()
 {
     uint64_t p;
@@ -155,6 +162,19 @@ __device__ __forceinline__ uint64_t sdesc_k_sw128(uint32_t saddr)
     d |= static_cast<uint64_t>(1024 >> 4) << 32;             // stride offset  [32,46)
     d |= static_cast<uint64_t>(1) << 46;                     // descriptor version (sm_100)
     d |= static_cast<uint64_t>(2) << 61;                     // 128-byte swizzle
+    return d;
+}
+
+// Same for a K-major tile stored with the 64-byte swizzle: rows of 64 bytes,
+// 8-row groups 512 bytes apart.
+__device__ __forceinline__ uint64_t sdesc_k_sw64(uint32_t saddr)
+{
+    uint64_t d = 0;
+    d |= static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4);   // start address  [0,14)
+    d |= static_cast<uint64_t>(1) << 16;                     // leading offset [16,30) (unused)
+    d |= static_cast<uint64_t>(512 >> 4) << 32;              // stride offset  [32,46)
+    d |= static_cast<uint64_t>(1) << 46;                     // descriptor version (sm_100)
+    d |= static_cast<uint64_t>(4) << 61;                     // 64-byte swizzle
     return d;
 }
 
