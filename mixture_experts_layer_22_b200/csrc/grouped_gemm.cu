@@ -55,7 +55,8 @@ struct GemmParams {
     int32_t *status;
     int32_t *counters;
     float *partials;
-    int stream_k;     // 0: whole tiles only
+    int stream_k;     // 0: whole tiles only; 1: stream-K the last 1-2 rounds;
+                      // 2: whole tiles unless the rounds would be < 90% full
 };
 
 template <int kMode, bool kSwap, bool kFp8, int kBN, bool kW8 = false>
@@ -281,6 +282,10 @@ __global__ void __launch_bounds__(Cfg<kMode, kSwap, kFp8, kBN, kW8>::kThreads, 1
     __shared__ volatile int s_abort;
     __shared__ int s_is_last;
     __shared__ float s_xchg[kMode == 0 && kSwap ? 16 * 64 : 1];
+    // normal order: per-warp staging of 32 rows x 64 bytes (80-byte pitch, no
+    // bank conflicts) so that the output is written as whole row segments
+    constexpr int kStagePitch = 80;
+    __shared__ __align__(16) uint8_t s_out_stage[kSwap ? 16 : C::kEpiWarps * 32 * kStagePitch];
     constexpr int kAN = kW8 ? C::kAStages : 1;
     __shared__ __align__(8) uint64_t s_a_full[kAN], s_a_empty[kAN];
 
@@ -358,7 +363,9 @@ __global__ void __launch_bounds__(Cfg<kMode, kSwap, kFp8, kBN, kW8>::kThreads, 1
     S.n_tiles = s_prefix[Et];
     S.KT = p.K / C::kKStage;
     S.G = gridDim.x;
-    if (!p.stream_k || S.n_tiles % S.G == 0) S.dp_tiles = S.n_tiles;
+    const bool full_enough = S.n_tiles >= S.G &&
+                             10 * S.n_tiles >= 9 * S.G * ((S.n_tiles + S.G - 1) / S.G);
+    if (!p.stream_k || S.n_tiles % S.G == 0 || (p.stream_k == 2 && full_enough)) S.dp_tiles = S.n_tiles;
     else if (S.n_tiles <= S.G) S.dp_tiles = 0;
     else S.dp_tiles = (S.n_tiles / S.G - 1) * S.G;
     S.sk_tiles = S.n_tiles - S.dp_tiles;
@@ -698,54 +705,83 @@ __global__ void __launch_bounds__(Cfg<kMode, kSwap, kFp8, kBN, kW8>::kThreads, 1
                                 __uint_as_float(v[j]) * sc;
                     }
                 } else if (kMode == 0) {
+                    // 32 features per chunk: h row segment of 64 (bf16) or 32 (E4M3) bytes
                     const int f0 = it.ft * 128;
-                    const bool valid = r < rows;
-                    for (int c0 = ch * (128 / kNch); c0 < (ch + 1) * (128 / kNch); c0 += 16) {
-                        uint32_t g[16], u[16];
+                    uint8_t *stg = s_out_stage + (warp - 2) * 32 * kStagePitch;
+                    const float inv_q = kFp8 ? 1.0f / p.qscale : 1.0f;
+                    for (int c0 = ch * (128 / kNch); c0 < (ch + 1) * (128 / kNch); c0 += 32) {
+                        uint32_t g[16], u[16], g2[16], u2[16];
                         tmem_ld16(tacc + c0, g);
                         tmem_ld16(tacc + 128 + c0, u);
+                        tmem_ld16(tacc + c0 + 16, g2);
+                        tmem_ld16(tacc + 128 + c0 + 16, u2);
                         tmem_wait_ld();
-                        if (valid) {
-                            float hv[16];
+                        float hv[32];
 #pragma unroll
-                            for (int j = 0; j < 16; ++j)
-                                hv[j] = silu_mul(__uint_as_float(g[j]) * sc, __uint_as_float(u[j]) * sc);
-                            const size_t o = static_cast<size_t>(row0 + r) * p.out_ld + f0 + c0;
-                            if (kFp8) {
+                        for (int j = 0; j < 16; ++j) {
+                            hv[j] = silu_mul(__uint_as_float(g[j]) * sc, __uint_as_float(u[j]) * sc);
+                            hv[16 + j] = silu_mul(__uint_as_float(g2[j]) * sc, __uint_as_float(u2[j]) * sc);
+                        }
+                        uint4 *wr = reinterpret_cast<uint4 *>(stg + lane * kStagePitch);
+                        if (kFp8) {
+#pragma unroll
+                            for (int j = 0; j < 2; ++j) {
                                 uint32_t w4[4];
 #pragma unroll
-                                for (int j = 0; j < 4; ++j)
-                                    w4[j] = e4m3_code(hv[4 * j] / p.qscale) | (e4m3_code(hv[4 * j + 1] / p.qscale) << 8) |
-                                            (e4m3_code(hv[4 * j + 2] / p.qscale) << 16) |
-                                            (e4m3_code(hv[4 * j + 3] / p.qscale) << 24);
-                                *reinterpret_cast<uint4 *>(static_cast<uint8_t *>(p.out) + o) =
-                                    make_uint4(w4[0], w4[1], w4[2], w4[3]);
-                            } else {
-                                uint32_t w8[8];
-#pragma unroll
-                                for (int j = 0; j < 8; ++j) w8[j] = pack_bf16x2(hv[2 * j], hv[2 * j + 1]);
-                                uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(p.out) + o);
-                                dst[0] = make_uint4(w8[0], w8[1], w8[2], w8[3]);
-                                dst[1] = make_uint4(w8[4], w8[5], w8[6], w8[7]);
+                                for (int i2 = 0; i2 < 4; ++i2) {
+                                    const int b = 16 * j + 4 * i2;
+                                    w4[i2] = e4m3_code(hv[b] * inv_q) | (e4m3_code(hv[b + 1] * inv_q) << 8) |
+                                             (e4m3_code(hv[b + 2] * inv_q) << 16) | (e4m3_code(hv[b + 3] * inv_q) << 24);
+                                }
+                                wr[j] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
                             }
+                        } else {
+#pragma unroll
+                            for (int j = 0; j < 4; ++j)
+                                wr[j] = make_uint4(pack_bf16x2(hv[8 * j], hv[8 * j + 1]), pack_bf16x2(hv[8 * j + 2], hv[8 * j + 3]),
+                                                   pack_bf16x2(hv[8 * j + 4], hv[8 * j + 5]), pack_bf16x2(hv[8 * j + 6], hv[8 * j + 7]));
                         }
+                        __syncwarp();
+                        constexpr int kSegLanes = kFp8 ? 2 : 4;          // 16-byte pieces per row segment
+                        constexpr int kRowsPerPass = 32 / kSegLanes;
+                        const size_t esz = kFp8 ? 1 : 2;
+#pragma unroll
+                        for (int ps = 0; ps < kSegLanes; ++ps) {
+                            const int rl = ps * kRowsPerPass + lane / kSegLanes;
+                            const int rg = q * 32 + rl;
+                            const uint4 val = *reinterpret_cast<const uint4 *>(stg + rl * kStagePitch + (lane % kSegLanes) * 16);
+                            if (rg < rows)
+                                *reinterpret_cast<uint4 *>(static_cast<uint8_t *>(p.out) +
+                                                           (static_cast<size_t>(row0 + rg) * p.out_ld + f0 + c0) * esz +
+                                                           (lane % kSegLanes) * 16) = val;
+                        }
+                        __syncwarp();
                     }
                 } else {
+                    // 16 fp32 columns per chunk: y row segment of 64 bytes
                     const int h0 = it.ft * 256;
-                    const bool valid = r < rows;
+                    uint8_t *stg = s_out_stage + (warp - 2) * 32 * kStagePitch;
                     for (int c0 = ch * (256 / kNch); c0 < (ch + 1) * (256 / kNch); c0 += 16) {
                         if (h0 + c0 >= p.n_feat) break;
                         uint32_t v[16];
                         ld_acc16(c0, v);
                         tmem_wait_ld();
-                        if (valid) {
-                            float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(p.out) +
-                                                                     static_cast<size_t>(row0 + r) * p.out_ld + h0 + c0);
+                        float4 *wr = reinterpret_cast<float4 *>(stg + lane * kStagePitch);
 #pragma unroll
-                            for (int j = 0; j < 4; ++j)
-                                dst[j] = make_float4(__uint_as_float(v[4 * j]) * sc, __uint_as_float(v[4 * j + 1]) * sc,
-                                                     __uint_as_float(v[4 * j + 2]) * sc, __uint_as_float(v[4 * j + 3]) * sc);
+                        for (int j = 0; j < 4; ++j)
+                            wr[j] = make_float4(__uint_as_float(v[4 * j]) * sc, __uint_as_float(v[4 * j + 1]) * sc,
+                                                __uint_as_float(v[4 * j + 2]) * sc, __uint_as_float(v[4 * j + 3]) * sc);
+                        __syncwarp();
+#pragma unroll
+                        for (int ps = 0; ps < 4; ++ps) {
+                            const int rl = ps * 8 + (lane >> 2);
+                            const int rg = q * 32 + rl;
+                            const float4 val = *reinterpret_cast<const float4 *>(stg + rl * kStagePitch + (lane & 3) * 16);
+                            if (rg < rows)
+                                *reinterpret_cast<float4 *>(static_cast<float *>(p.out) +
+                                                            static_cast<size_t>(row0 + rg) * p.out_ld + h0 + c0 + (lane & 3) * 4) = val;
                         }
+                        __syncwarp();
                     }
                 }
                 tc_fence_before();
@@ -941,7 +977,9 @@ static cudaError_t run_gemm(const moe_shape_t &s, const GemmArgs &a, cudaStream_
     p.status = a.status;
     p.counters = a.counters;
     p.partials = a.partials;
-    p.stream_k = 1;
+    // decode tiles split cheaply (few token columns); prefill tiles carry
+    // 128 KB of fp32 partials, so whole tiles are preferred there
+    p.stream_k = kSwap ? 1 : 2;
     cudaError_t err = cudaMemsetAsync(a.counters, 0, 2 * kMaxCtas * sizeof(int32_t), st);
     if (err != cudaSuccess) return err;
     kern<<<sm_count(), Cf::kThreads, Cf::kDynSmem, st>>>(tm_w, tm_x, p);
