@@ -42,9 +42,9 @@ def workload_desc(wl) -> str:
     return (f"{wl.name}: T={wl.T} H={wl.H} I={wl.I} E={wl.E} top-{wl.k} {gate}{sh}, {dt}")
 
 
-def config_of(wl, parallelism: str) -> dict:
+def config_of(wl, parallelism: str, launch: str = "") -> dict:
     return {"workload": workload_desc(wl), "T": wl.T, "H": wl.H, "I": wl.I, "E": wl.E, "k": wl.k,
-            "n_shared": wl.n_shared, "parallelism": parallelism,
+            "n_shared": wl.n_shared, "parallelism": parallelism, "launch": launch,
             "l2": "no flush: the step streams all active expert weights (GBs) through the 126 MB L2",
             "inputs": "seeded synthetic (seed 0), resident in HBM before timing"}
 
@@ -219,10 +219,29 @@ def ours_main(args, wl):
     a2 = float(args.a2) if args.a2 is not None else static_hidden_scale(wl)
     out = torch.empty((wl.T, wl.H), dtype=torch.bfloat16, device=dev)
     ws = moe.workspace(shape, device=dev)
-    stream = torch.cuda.current_stream(dev)
+    stream = torch.cuda.Stream(dev)        # graphs cannot be captured on the legacy default stream
+    torch.cuda.set_stream(stream)
+
+    def call():
+        moe.fused_forward(shape, x, logits, w13, s13, w2, s2, a1, a2, out, ws, stream)
+
+    # one layer call captured into a CUDA graph (the library launches no host
+    # syncs, so the whole 6-7 kernel sequence is capturable); replaying it
+    # removes the per-call host cost from the timed region
+    graph = None
+    if not args.no_graph:
+        call()
+        torch.cuda.synchronize(dev)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=stream):
+            call()
+        torch.cuda.synchronize(dev)
 
     def step():
-        moe.fused_forward(shape, x, logits, w13, s13, w2, s2, a1, a2, out, ws, stream)
+        if graph is not None:
+            graph.replay()
+        else:
+            call()
 
     # routing facts for the roofline: distinct active experts and routed rows
     E_t = wl.E + wl.n_shared
@@ -240,6 +259,8 @@ def ours_main(args, wl):
 
     for _ in range(args.warmup):
         step()
+    torch.cuda.synchronize(dev)
+    call()
     torch.cuda.synchronize(dev)
     launches_per_step = moe.last_launch_count()
     st = moe.device_status(ws, stream)
@@ -322,10 +343,21 @@ def ours_main(args, wl):
     dx = torch.empty_like(x)
     dl = torch.empty_like(logits)
 
+    e2e_graph = None
+    if not args.no_graph:
+        torch.cuda.synchronize(dev)
+        e2e_graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(e2e_graph, stream=stream):
+            moe.fused_forward(shape, dx, dl, w13, s13, w2, s2, a1, a2, out, ws, stream)
+        torch.cuda.synchronize(dev)
+
     def e2e_step():
         dx.copy_(hx, non_blocking=True)
         dl.copy_(hl, non_blocking=True)
-        moe.fused_forward(shape, dx, dl, w13, s13, w2, s2, a1, a2, out, ws, stream)
+        if e2e_graph is not None:
+            e2e_graph.replay()
+        else:
+            moe.fused_forward(shape, dx, dl, w13, s13, w2, s2, a1, a2, out, ws, stream)
         ho.copy_(out, non_blocking=True)
 
     for _ in range(args.warmup):
@@ -351,7 +383,9 @@ def ours_main(args, wl):
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": {(0, 0): "bf16", (1, 1): "e4m3", (1, 0): "e4m3w-bf16a"}[(wl.wdtype, wl.adtype)],
-        "data": "synthetic", "config": config_of(wl, f"replicas x{world}" if world > 1 else "1 GPU"),
+        "data": "synthetic",
+        "config": config_of(wl, f"replicas x{world}" if world > 1 else "1 GPU",
+                            "direct launches" if args.no_graph else "CUDA graph of one moe_fused_forward per step"),
         "hbm_gbs": layer_bytes / (ms_per_step * 1e-3) / 1e9, "tflops": flops / (ms_per_step * 1e-3) / 1e12,
         "active_experts": active,
         "roofline": roof,
@@ -383,6 +417,7 @@ def main():
                     help="static hidden-activation scale (FP8 activations; default: the calibrated golden value)")
     ap.add_argument("--ref-budget", type=float, default=15.0, help="seconds of host time per oracle sample")
     ap.add_argument("--no-cpu", action="store_true", help="skip the cpu_baseline leg")
+    ap.add_argument("--no-graph", action="store_true", help="launch each step directly instead of replaying a CUDA graph")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

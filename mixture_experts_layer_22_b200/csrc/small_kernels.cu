@@ -246,6 +246,84 @@ __global__ void __launch_bounds__(1024) align_scatter_kernel(const int32_t *__re
     }
 }
 
+// All routed rows in one block (R <= 1024, every decode batch here): count,
+// scan, pad and place in a single launch, with the histogram, the offsets and
+// the per-warp counts in shared memory.  Same result as the two-kernel path.
+__global__ void __launch_bounds__(1024) align_single_kernel(const int32_t *__restrict__ ids, int R, int T,
+                                                            int E, int n_shared, int pad, int32_t *counts,
+                                                            int32_t *offsets, int32_t *sorted_rows,
+                                                            int32_t *inv, Ctrl *ctrl)
+{
+    extern __shared__ int32_t sm_al[];
+    const int Et = E + n_shared;
+    int32_t *hist = sm_al;                 // [Et]: counts, then segment starts
+    int32_t *wc = sm_al + Et;              // [32 warps][Et]
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    for (int i = tid; i < Et * 33; i += blockDim.x) sm_al[i] = 0;
+    __syncthreads();
+    const int f = tid;
+    int e = f < R ? ids[f] : -1;
+    const bool valid = e >= 0 && e < E;
+    if (f < R && !valid) set_status(&ctrl->status, MOE_ERR_DEVICE_CHECK);
+    if (!valid) e = -1;
+    const unsigned same = __match_any_sync(0xffffffffu, e);
+    const int rank = __popc(same & ((1u << lane) - 1u));
+    if (valid && rank == 0) {
+        wc[warp * Et + e] = __popc(same);
+        atomicAdd(&hist[e], __popc(same));
+    }
+    __syncthreads();
+    for (int x = tid; x < Et; x += blockDim.x) {
+        const int c = x < E ? hist[x] : T;
+        counts[x] = c;
+        hist[x] = (c + pad - 1) / pad * pad;
+        int run = 0;                                     // exclusive prefix over warps
+        for (int q = 0; q < 32; ++q) {
+            const int v = wc[q * Et + x];
+            wc[q * Et + x] = run;
+            run += v;
+        }
+    }
+    __syncthreads();
+    if (tid < 32) {                                      // exclusive scan of padded sizes
+        const int per = (Et + 31) / 32;
+        const int lo = min(Et, tid * per), hi = min(Et, lo + per);
+        int sum = 0;
+        for (int x = lo; x < hi; ++x) sum += hist[x];
+        int inc = sum;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(0xffffffffu, inc, o);
+            if (tid >= o) inc += v;
+        }
+        int run = inc - sum;
+        for (int x = lo; x < hi; ++x) {
+            const int sz = hist[x];
+            offsets[x] = run;
+            hist[x] = run;
+            run += sz;
+        }
+        if (tid == 31) offsets[Et] = inc;
+    }
+    __syncthreads();
+    for (int x = tid; x < Et; x += blockDim.x) {         // pad slots
+        const int start = hist[x], c = counts[x];
+        const int end = start + (c + pad - 1) / pad * pad;
+        for (int q = start + c; q < end; ++q) sorted_rows[q] = -1;
+    }
+    for (int sh = 0; sh < n_shared; ++sh)
+        for (int t = tid; t < T; t += blockDim.x) sorted_rows[hist[E + sh] + t] = R + sh * T + t;
+    if (f < R) {
+        if (valid) {
+            const int slot = hist[e] + wc[warp * Et + e] + rank;
+            sorted_rows[slot] = f;
+            inv[f] = slot;
+        } else {
+            inv[f] = -1;
+        }
+    }
+}
+
 cudaError_t launch_align(const moe_shape_t &s, const int32_t *ids, int32_t *counts,
                          int32_t *offsets, int32_t *sorted_rows, int32_t *inv, int32_t *chunk_hist,
                          int32_t *chunk_base, Ctrl *ctrl, cudaStream_t st, int *launches)
@@ -256,7 +334,15 @@ cudaError_t launch_align(const moe_shape_t &s, const int32_t *ids, int32_t *coun
     if (!attr_done) {
         cudaFuncSetAttribute(align_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              32 * kMaxExpertsTotal * 4);
+        cudaFuncSetAttribute(align_single_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             33 * kMaxExpertsTotal * 4);
         attr_done = true;
+    }
+    if (nb == 1) {
+        align_single_kernel<<<1, kAlignChunk, 33 * Et * sizeof(int32_t), st>>>(ids, R, s.T, s.E, s.n_shared, s.pad,
+                                                                            counts, offsets, sorted_rows, inv, ctrl);
+        *launches += 1;
+        return cudaGetLastError();
     }
     cudaError_t err = cudaMemsetAsync(&ctrl->ticket, 0, sizeof(int32_t), st);
     if (err != cudaSuccess) return err;
@@ -278,24 +364,26 @@ __global__ void __launch_bounds__(256) gather_kernel(const uint4 *__restrict__ x
 {
     const int lane = threadIdx.x & 31;
     const int nvec = H / 8;                       // 8 bf16 per 16 bytes
+    const int nchunk = (nvec + 31) / 32;          // 512-byte chunks per row
     const int total = offsets[Et];
     const int R = T * k;
-    for (int s = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; s < total;
-         s += (gridDim.x * blockDim.x) >> 5) {
+    for (long long item = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; item < static_cast<long long>(total) * nchunk;
+         item += (gridDim.x * blockDim.x) >> 5) {
+        const int s = static_cast<int>(item / nchunk);
+        const int v = static_cast<int>(item % nchunk) * 32 + lane;
         const int f = sorted_rows[s];
         const int t = f < 0 ? -1 : (f < R ? f / k : (f - R) % T);
+        if (v >= nvec) continue;
         if (!kQuant) {
             uint4 *dst = reinterpret_cast<uint4 *>(xp) + static_cast<size_t>(s) * nvec;
             const uint4 *src = x + static_cast<size_t>(t < 0 ? 0 : t) * nvec;
-            for (int v = lane; v < nvec; v += 32) dst[v] = t < 0 ? make_uint4(0, 0, 0, 0) : __ldg(src + v);
+            dst[v] = t < 0 ? make_uint4(0, 0, 0, 0) : __ldg(src + v);
         } else {
             uint2 *dst = reinterpret_cast<uint2 *>(xp) + static_cast<size_t>(s) * nvec;
             const uint4 *src = x + static_cast<size_t>(t < 0 ? 0 : t) * nvec;
-            for (int v = lane; v < nvec; v += 32) {
-                if (t < 0) {
-                    dst[v] = make_uint2(0, 0);
-                    continue;
-                }
+            if (t < 0) {
+                dst[v] = make_uint2(0, 0);
+            } else {
                 const uint4 d = __ldg(src + v);
                 const uint32_t wv[4] = {d.x, d.y, d.z, d.w};
                 uint32_t q[2] = {0, 0};
@@ -317,7 +405,7 @@ cudaError_t launch_gather(const moe_shape_t &s, const void *x, const int32_t *so
                           cudaStream_t st)
 {
     const int Et = s.E + s.n_shared;
-    const int64_t warps = max_rows;
+    const int64_t warps = max_rows * ((s.H / 8 + 31) / 32);
     int blocks = static_cast<int>((warps + 7) / 8);
     if (blocks > 148 * 16) blocks = 148 * 16;
     if (blocks < 1) blocks = 1;
@@ -348,7 +436,8 @@ __global__ void __launch_bounds__(256) combine_kernel(const float4 *__restrict__
         s_w[threadIdx.x] = w[static_cast<size_t>(t) * k + threadIdx.x];
     }
     __syncthreads();
-    for (int c = threadIdx.x; c < n4; c += blockDim.x) {
+    // block (t, y) owns 4-column groups [y*256, (y+1)*256) of token t
+    for (int c = blockIdx.y * blockDim.x + threadIdx.x; c < n4; c += gridDim.y * blockDim.x) {
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
         for (int j = 0; j < k; ++j) {
             const int slot = s_slot[j];
@@ -379,8 +468,9 @@ __global__ void __launch_bounds__(256) combine_kernel(const float4 *__restrict__
 cudaError_t launch_combine(const moe_shape_t &s, const float *y, const float *w,
                            const int32_t *inv, const int32_t *offsets, void *out, cudaStream_t st)
 {
-    combine_kernel<<<s.T, 256, 0, st>>>(reinterpret_cast<const float4 *>(y), w, inv, offsets, s.H,
-                                        s.k, s.E, s.n_shared, static_cast<uint2 *>(out));
+    const dim3 grid(s.T, (s.H / 4 + 255) / 256);
+    combine_kernel<<<grid, 256, 0, st>>>(reinterpret_cast<const float4 *>(y), w, inv, offsets, s.H,
+                                         s.k, s.E, s.n_shared, static_cast<uint2 *>(out));
     return cudaGetLastError();
 }
 
