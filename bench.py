@@ -171,6 +171,23 @@ def measured_peaks():
         return 6650.0, 1590.0, 1400.0, "fallback"
 
 
+def captured_traffic(wl, which: str):
+    """DRAM bytes per launch of a grouped GEMM from the committed ncu capture
+    (profiles/traffic.json), or None when no capture exists for this workload
+    or the kernel source has changed since it was taken."""
+    import hashlib
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+            t = json.load(f)
+        with open(os.path.join(ROOT, "mixture_experts_layer_22_b200", "csrc", "grouped_gemm.cu"), "rb") as f:
+            sha = hashlib.sha256(f.read()).hexdigest()
+    except (OSError, ValueError):
+        return None
+    if sha != t.get("source_sha256"):
+        return None
+    return t.get("kernels", {}).get(f"{wl.name} T={wl.T} {which}")
+
+
 def static_hidden_scale(wl) -> float:
     """The oracle-calibrated static E4M3 scale of h (tests/golden), else 1."""
     if wl.adtype != syn.E4M3:
@@ -330,7 +347,8 @@ def ours_main(args, wl):
         peak = tc_burst * (2.0 if wl.adtype == syn.E4M3 else 1.0)
         roof = {"bound": "tensor", "achieved": g1_flops / (t_g1 * 1e-3) / 1e12, "peak": peak,
                 "unit": "TFLOP/s", "algorithmic_flops": g1_flops}
-    roof.update({"frac": roof["achieved"] / roof["peak"], "peak_kind": peak_kind, "traffic": None,
+    roof.update({"frac": roof["achieved"] / roof["peak"], "peak_kind": peak_kind,
+                 "traffic": captured_traffic(wl, "gemm1"),
                  "kernel": "grouped_gemm (gate/up + SwiGLU)", "ms": t_g1, "down_ms": t_g2,
                  "down_gbs": g2_bytes / (t_g2 * 1e-3) / 1e9,
                  "down_tflops": 2.0 * wl.H * wl.I * real_rows / (t_g2 * 1e-3) / 1e12})
