@@ -56,6 +56,24 @@ def dist_env():
     return ws, rank, local
 
 
+def aggregate_over_ranks(ms_local: float, tokens_per_rank: int, steps: int, dist_mod=None):
+    """Slowest rank's timed-region milliseconds and the whole-job tokens/s:
+    every rank contributes `tokens_per_rank * steps` tokens, the job takes as
+    long as its slowest rank.  With dist_mod (torch.distributed, initialised)
+    the max is an all-reduce over the process group; every rank returns the
+    same numbers."""
+    import torch
+    world = 1
+    ms = float(ms_local)
+    if dist_mod is not None and dist_mod.is_initialized():
+        world = dist_mod.get_world_size()
+        dev = torch.device("cuda", torch.cuda.current_device()) if dist_mod.get_backend() == "nccl" else "cpu"
+        t = torch.tensor([ms], dtype=torch.float64, device=dev)
+        dist_mod.all_reduce(t, op=dist_mod.ReduceOp.MAX)
+        ms = float(t.item())
+    return ms, world * tokens_per_rank * steps / (ms / 1e3)
+
+
 def weight_bytes_per_expert(wl) -> int:
     esz = 2 if wl.wdtype == syn.BF16 else 1
     return 3 * wl.H * wl.I * esz
@@ -299,13 +317,8 @@ def ours_main(args, wl):
     if world > 1:
         dist.barrier()
     clk = clocks.stop()
-    ms = ev0.elapsed_time(ev1)
-    if world > 1:
-        t = torch.tensor([ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms, value = aggregate_over_ranks(ev0.elapsed_time(ev1), wl.T, args.steps, dist if world > 1 else None)
     ms_per_step = ms / args.steps
-    value = world * wl.T * args.steps / (ms / 1e3)
 
     # per-kernel device time of the two expert GEMMs (same inputs, step-wise calls)
     xp = torch.empty((moe.max_rows(shape), wl.H * (1 if wl.adtype else 2)), dtype=torch.uint8, device=dev)
@@ -390,12 +403,7 @@ def ours_main(args, wl):
         stream.synchronize()
     e1.record(stream)
     torch.cuda.synchronize(dev)
-    ems = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([ems], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ems = float(t.item())
-    e2e_val = world * wl.T * args.steps / (ems / 1e3)
+    ems, e2e_val = aggregate_over_ranks(e0.elapsed_time(e1), wl.T, args.steps, dist if world > 1 else None)
 
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
