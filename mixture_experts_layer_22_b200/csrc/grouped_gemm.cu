@@ -287,7 +287,7 @@ __global__ void __launch_bounds__(Cfg<kMode, kSwap, kFp8, kBN, kW8>::kThreads, 1
     constexpr int kStagePitch = 80;
     __shared__ __align__(16) uint8_t s_out_stage[kSwap ? 16 : C::kEpiWarps * 32 * kStagePitch];
     constexpr int kAN = kW8 ? C::kAStages : 1;
-    __shared__ __align__(8) uint64_t s_a_full[kAN], s_a_empty[kAN];
+    __shared__ __align__(8) uint64_t s_a_full[kAN];
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int Et = p.E_tot;
@@ -310,10 +310,8 @@ __global__ void __launch_bounds__(Cfg<kMode, kSwap, kFp8, kBN, kW8>::kThreads, 1
         mbar_init(smem_u32(&s_drain), 1);
         mbar_init(smem_u32(&s_drain2), 1);
         if (kW8) {
-            for (int i = 0; i < kAN; ++i) {                    // one barrier pair per slab pair
+            for (int i = 0; i < kAN; ++i)                      // one barrier per slab pair
                 mbar_init(smem_u32(&s_a_full[i]), 4);         // the four warps of a converter group
-                mbar_init(smem_u32(&s_a_empty[i]), 2);        // both MMA warps
-            }
         }
         fence_mbar_init();
         prefetch_tmap(&tm_w);
@@ -422,7 +420,9 @@ __global__ void __launch_bounds__(Cfg<kMode, kSwap, kFp8, kBN, kW8>::kThreads, 1
         // j = g, g+2, ...), so two stages are converted at once.  Warp w
         // covers the 32 weight rows of its tensor-memory lane quarter (w % 4):
         // thread = one row, both K halves (2 x 64 codes -> 2 x 32 packed
-        // columns), stored into slab pair j % 4 with tcgen05.st.
+        // columns), stored into slab pair j % 4 with tcgen05.st.  Slab pair
+        // j % 4 is free once stage j-4 has been released (its release needs
+        // both MMA warps' commits, i.e. its MMAs have completed).
         const int group = (warp - 6) >> 2;
         const int q = warp & 3;
         const int r = q * 32 + lane;
@@ -437,9 +437,13 @@ __global__ void __launch_bounds__(Cfg<kMode, kSwap, kFp8, kBN, kW8>::kThreads, 1
             for (int kk = it.kb; kk < it.ke; ++kk, ++j) {
                 if ((j & 1) == group) {
                     const int pr = j & 3;
-                    const uint32_t aph = static_cast<uint32_t>(j >> 2) & 1u;
-                    if (!mbar_wait(smem_u32(&s_full[stage]), phase, &s_abort) ||
-                        !mbar_wait(smem_u32(&s_a_empty[pr]), aph ^ 1u, &s_abort)) {
+                    bool got = mbar_wait(smem_u32(&s_full[stage]), phase, &s_abort);
+                    if (got && j >= 4) {
+                        const int jp = j - 4;
+                        got = mbar_wait(smem_u32(&s_empty[jp % C::kStages]),
+                                        static_cast<uint32_t>(jp / C::kStages) & 1u, &s_abort);
+                    }
+                    if (!got) {
                         ok = false;
                         break;
                     }
@@ -472,7 +476,7 @@ __global__ void __launch_bounds__(Cfg<kMode, kSwap, kFp8, kBN, kW8>::kThreads, 1
         if (lane == 0) {
             const int hh = warp == 1 ? 0 : 1;
             int stage = 0, acc = 0, j = 0;
-            uint32_t phase = 0, acc_phase = 0;
+            uint32_t acc_phase = 0;
             ItemIter I;
             iter_init(I, S, blockIdx.x);
             Item it;
@@ -486,10 +490,9 @@ __global__ void __launch_bounds__(Cfg<kMode, kSwap, kFp8, kBN, kW8>::kThreads, 1
                 const uint32_t idesc = idesc_make(1u, 128, n);
                 for (int kk = it.kb; kk < it.ke; ++kk, ++j) {
                     const int pr = j & 3;
-                    // the activation rows landed with the stage (full); the
-                    // converted weight slabs with the pair's a_full
-                    if (!mbar_wait(smem_u32(&s_full[stage]), phase, &s_abort) ||
-                        !mbar_wait(smem_u32(&s_a_full[pr]), static_cast<uint32_t>(j >> 2) & 1u, &s_abort)) {
+                    // the converters arrive on a_full only after observing the
+                    // stage's full barrier, so the activation rows have landed too
+                    if (!mbar_wait(smem_u32(&s_a_full[pr]), static_cast<uint32_t>(j >> 2) & 1u, &s_abort)) {
                         ok = false;
                         break;
                     }
@@ -501,12 +504,8 @@ __global__ void __launch_bounds__(Cfg<kMode, kSwap, kFp8, kBN, kW8>::kThreads, 1
                     for (int s4 = 0; s4 < 4; ++s4)
                         mma_bf16_tmem_a(d, ta + s4 * 8, bd0 + static_cast<uint64_t>(s4 * 2), idesc,
                                         (kk > it.kb || s4 > 0) ? 1u : 0u);
-                    mma_commit(smem_u32(&s_a_empty[pr]));
                     mma_commit(smem_u32(&s_empty[stage]));
-                    if (++stage == C::kStages) {
-                        stage = 0;
-                        phase ^= 1u;
-                    }
+                    if (++stage == C::kStages) stage = 0;
                 }
                 if (!ok) break;
                 mma_commit(smem_u32(&s_tfull[acc]));
