@@ -55,8 +55,13 @@ struct GemmParams {
     int32_t *status;
     int32_t *counters;
     float *partials;
-    int stream_k;     // 0: whole tiles only; 1: stream-K the last 1-2 rounds;
-                      // 2: whole tiles unless the rounds would be < 90% full
+    int stream_k;     // 0: whole tiles only.  Otherwise whole tiles for all but the
+                      // last one or two rounds, which are split into equal K-step ranges
+                      // (stream-K, each tile shared by at most ~2 CTAs), except that whole
+                      // tiles are used throughout when the last round is full enough:
+                      // 1 (HBM-bound decode): >= 70% of the CTAs busy (an idle SM costs
+                      //   little while the others keep HBM saturated);
+                      // 2 (tensor-bound prefill): rounds >= 90% full on average.
 };
 
 template <int kMode, bool kSwap, bool kFp8, int kBN, bool kW8 = false>
@@ -281,6 +286,7 @@ __global__ void __launch_bounds__(Cfg<kMode, kSwap, kFp8, kBN, kW8>::kThreads, 1
     __shared__ uint32_t s_tmem_base;
     __shared__ volatile int s_abort;
     __shared__ int s_is_last;
+    __shared__ int s_slot_of[kMaxCtas];     // stream-K fixup: partial slot of each contributor
     __shared__ float s_xchg[kMode == 0 && kSwap ? 16 * 64 : 1];
     // normal order: per-warp staging of 32 rows x 64 bytes (80-byte pitch, no
     // bank conflicts) so that the output is written as whole row segments
@@ -361,10 +367,12 @@ __global__ void __launch_bounds__(Cfg<kMode, kSwap, kFp8, kBN, kW8>::kThreads, 1
     S.n_tiles = s_prefix[Et];
     S.KT = p.K / C::kKStage;
     S.G = gridDim.x;
+    const int rem = S.n_tiles % S.G;
     const bool full_enough = S.n_tiles >= S.G &&
                              10 * S.n_tiles >= 9 * S.G * ((S.n_tiles + S.G - 1) / S.G);
-    if (!p.stream_k || S.n_tiles % S.G == 0 || (p.stream_k == 2 && full_enough)) S.dp_tiles = S.n_tiles;
-    else if (S.n_tiles <= S.G) S.dp_tiles = 0;
+    if (!p.stream_k || rem == 0) S.dp_tiles = S.n_tiles;
+    else if (S.n_tiles < S.G) S.dp_tiles = 0;
+    else if ((p.stream_k == 1 && 10 * rem >= 7 * S.G) || (p.stream_k == 2 && full_enough)) S.dp_tiles = S.n_tiles;
     else S.dp_tiles = (S.n_tiles / S.G - 1) * S.G;
     S.sk_tiles = S.n_tiles - S.dp_tiles;
     S.sk_total = static_cast<long long>(S.sk_tiles) * S.KT;
@@ -812,10 +820,14 @@ __global__ void __launch_bounds__(Cfg<kMode, kSwap, kFp8, kBN, kW8>::kThreads, 1
                 named_bar_sync(1, C::kEpiThreads);
                 if (s_is_last) {
                     __threadfence();
-                    auto slot_of = [&](int c) -> const float * {
+                    // partial slot of every contributing CTA, once (64-bit divisions)
+                    for (int c = c_first + etid; c <= c_last; c += C::kEpiThreads) {
                         const int first_tile = static_cast<int>(sk_begin(c, S) / S.KT);
-                        const int sidx = 2 * c + (first_tile == it.sk_tile ? 0 : 1);
-                        return p.partials + static_cast<size_t>(sidx) * 128 * C::kAccCols;
+                        s_slot_of[c - c_first] = 2 * c + (first_tile == it.sk_tile ? 0 : 1);
+                    }
+                    named_bar_sync(1, C::kEpiThreads);
+                    auto slot_of = [&](int c) -> const float * {
+                        return p.partials + static_cast<size_t>(s_slot_of[c - c_first]) * 128 * C::kAccCols;
                     };
                     if (kSwap && kMode == 0) {
                         const int f0 = it.ft * 64;
