@@ -189,16 +189,27 @@ def measured_peaks():
         return 6650.0, 1590.0, 1400.0, "fallback"
 
 
+KERNEL_SOURCES = ("grouped_gemm.cu", "ptx.cuh", "common.cuh")
+
+
+def kernel_source_sha256() -> str:
+    """sha256 over the grouped GEMM's source files, concatenated in order."""
+    import hashlib
+    h = hashlib.sha256()
+    for name in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, "mixture_experts_layer_22_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
 def captured_traffic(wl, which: str):
     """DRAM bytes per launch of a grouped GEMM from the committed ncu capture
     (profiles/traffic.json), or None when no capture exists for this workload
     or the kernel source has changed since it was taken."""
-    import hashlib
     try:
         with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
             t = json.load(f)
-        with open(os.path.join(ROOT, "mixture_experts_layer_22_b200", "csrc", "grouped_gemm.cu"), "rb") as f:
-            sha = hashlib.sha256(f.read()).hexdigest()
+        sha = kernel_source_sha256()
     except (OSError, ValueError):
         return None
     if sha != t.get("source_sha256"):

@@ -26,6 +26,36 @@ __device__ __forceinline__ void set_status(int32_t *status, int32_t code)
     atomicCAS(status, 0, code);
 }
 
+// Programmatic dependent launch.  Inside moe_fused_forward each kernel after
+// the first is launched while its predecessor still runs.  Every kernel calls
+// grid_dep_wait() (the predecessor grid has completed and its writes are
+// visible) before it writes anything (other than an atomic first-error
+// status) and before it reads what its predecessor writes; only then does it let its own successor launch.  So
+// when a kernel starts, every kernel two or more places before it has
+// completed: the grouped GEMMs read the segment offsets (written by align)
+// and prefetch weights before they wait.  Both calls are no-ops in a kernel
+// launched without the attribute.
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+// Launch with the programmatic-stream-serialisation attribute when `pdl`.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_kernel(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                          bool pdl, Args... args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
+
 // Workspace carving (host side), every region 256-byte aligned.
 struct WsLayout {
     size_t ctrl, ids, w, counts, offsets, chunk_hist, chunk_base, sorted_rows, inv;
@@ -49,15 +79,19 @@ int validate_shape(const moe_shape_t *s, bool need_gemm);
 // ---- launchers (return cudaError_t of the launch) ----
 cudaError_t launch_route(const moe_shape_t &s, const float *logits, int32_t *ids, float *w,
                          cudaStream_t st);
+// `chained`: launched by moe_fused_forward after its first kernel (PDL
+// launch; the control words and GEMM tile counters were zeroed at the start
+// of the call)
 cudaError_t launch_align(const moe_shape_t &s, const int32_t *ids, int32_t *counts,
                          int32_t *offsets, int32_t *sorted_rows, int32_t *inv, int32_t *chunk_hist,
-                         int32_t *chunk_base, Ctrl *ctrl, cudaStream_t st, int *launches);
+                         int32_t *chunk_base, Ctrl *ctrl, cudaStream_t st, int *launches,
+                         bool chained = false);
 cudaError_t launch_gather(const moe_shape_t &s, const void *x, const int32_t *sorted_rows,
                           const int32_t *offsets, float a1, void *xp, int64_t max_rows,
-                          cudaStream_t st);
+                          cudaStream_t st, bool chained = false);
 cudaError_t launch_combine(const moe_shape_t &s, const float *y, const float *w,
                            const int32_t *inv, const int32_t *offsets, void *out,
-                           cudaStream_t st);
+                           cudaStream_t st, bool chained = false);
 
 struct GemmArgs {
     int mode;                 // 0: gate/up + SwiGLU, 1: down projection
@@ -71,6 +105,7 @@ struct GemmArgs {
     int32_t *counters;
     float *partials;
     int64_t max_rows;
+    bool chained;             // PDL launch; counters already zero
 };
 cudaError_t launch_grouped_gemm(const moe_shape_t &s, const GemmPlan &p, const GemmArgs &a,
                                 cudaStream_t st, int *launches, int *host_err);

@@ -55,6 +55,8 @@ struct GemmParams {
     int32_t *status;
     int32_t *counters;
     float *partials;
+    int pdl;          // launched as a programmatic dependent: prefetch the first weight
+                      // stages into L2 before waiting for the previous kernel
     int stream_k;     // 0: whole tiles only.  Otherwise whole tiles for all but the
                       // last one or two rounds, which are split into equal K-step ranges
                       // (stream-K, each tile shared by at most ~2 CTAs), except that whole
@@ -329,7 +331,9 @@ __global__ void __launch_bounds__(Cfg<kMode, kSwap, kFp8, kBN, kW8>::kThreads, 1
     }
     const int n_ft = (p.n_feat + C::kFeatTile - 1) / C::kFeatTile;
     if (warp == 2) {
-        for (int e = lane; e <= Et; e += 32) s_off[e] = p.offsets[e];
+        // L2 load: under PDL this runs before grid_dep_wait(); the offsets
+        // come from the align kernel, which has completed by then
+        for (int e = lane; e <= Et; e += 32) s_off[e] = __ldcg(p.offsets + e);
         __syncwarp();
         const int per = (Et + 31) / 32;
         const int lo = min(Et, lane * per), hi = min(Et, lo + per);
@@ -377,6 +381,34 @@ __global__ void __launch_bounds__(Cfg<kMode, kSwap, kFp8, kBN, kW8>::kThreads, 1
     S.sk_tiles = S.n_tiles - S.dp_tiles;
     S.sk_total = static_cast<long long>(S.sk_tiles) * S.KT;
     S.sk_ctas = static_cast<int>(S.sk_total < S.G ? S.sk_total : S.G);
+
+    // ---- programmatic dependent launch ----
+    // Everything above reads only the offsets.  The weights are never written
+    // by an earlier kernel, so the producer first pulls the opening stages of
+    // this CTA's weight stream into L2; every thread then waits for the
+    // previous kernel (which wrote the activations this kernel reads) before
+    // touching anything else in global memory.
+    if (warp == 0 && lane == 0 && p.pdl) {
+        constexpr int kHalf = kSwap ? 64 : 128;   // weight rows per gate/up half-tile
+        ItemIter I;
+        iter_init(I, S, blockIdx.x);
+        Item it;
+        int n = 0;
+        while (n < C::kStages && iter_next<C::kRowsTile>(I, S, s_prefix, s_off, Et, n_ft, it)) {
+            const int wbase = it.e * p.w_rows;
+            for (int kk = it.kb; kk < it.ke && n < C::kStages; ++kk, ++n) {
+                const int kx = kk * C::kKStage;
+                if (kMode == 0) {
+                    tma_prefetch_l2_2d(&tm_w, kx, wbase + it.ft * kHalf);
+                    tma_prefetch_l2_2d(&tm_w, kx, wbase + p.n_feat + it.ft * kHalf);
+                } else {
+                    tma_prefetch_l2_2d(&tm_w, kx, wbase + it.ft * 2 * kHalf);
+                }
+            }
+        }
+    }
+    grid_dep_wait();
+    grid_dep_launch();
 
 
     if (kW8 && warp == 0) {
@@ -991,10 +1023,12 @@ static cudaError_t run_gemm(const moe_shape_t &s, const GemmArgs &a, cudaStream_
     // decode tiles split cheaply (few token columns); prefill tiles carry
     // 128 KB of fp32 partials, so whole tiles are preferred there
     p.stream_k = kSwap ? 1 : 2;
-    cudaError_t err = cudaMemsetAsync(a.counters, 0, 2 * kMaxCtas * sizeof(int32_t), st);
-    if (err != cudaSuccess) return err;
-    kern<<<sm_count(), Cf::kThreads, Cf::kDynSmem, st>>>(tm_w, tm_x, p);
-    return cudaGetLastError();
+    p.pdl = a.chained ? 1 : 0;
+    if (!a.chained) {
+        cudaError_t err = cudaMemsetAsync(a.counters, 0, 2 * kMaxCtas * sizeof(int32_t), st);
+        if (err != cudaSuccess) return err;
+    }
+    return launch_kernel(kern, dim3(sm_count()), dim3(Cf::kThreads), Cf::kDynSmem, st, a.chained, tm_w, tm_x, p);
 }
 
 int gemm_acc_cols(const GemmPlan &p) { return p.swap ? p.bn : 256; }

@@ -68,6 +68,9 @@ bool ws_layout(const moe_shape_t &s, WsLayout &L)
     const size_t ab = s.adtype == MOE_E4M3 ? 1 : 2;
     size_t o = 0;
     L.ctrl = o;        o += up256(sizeof(Ctrl));
+    // stream-K tile counters right after the control words (one memset
+    // clears both): GEMM1 uses the first half, GEMM2 the second
+    L.counters = o;    o += up256(4 * kMaxCtas * 4);
     L.ids = o;         o += up256(R * 4);
     L.w = o;           o += up256(R * 4);
     L.counts = o;      o += up256(Et * 4);
@@ -79,7 +82,6 @@ bool ws_layout(const moe_shape_t &s, WsLayout &L)
     L.xp = o;          o += up256(L.max_rows * s.H * ab);
     L.h = o;           o += up256(L.max_rows * s.I * ab);
     L.y = o;           o += up256(L.max_rows * s.H * 4);
-    L.counters = o;    o += up256(2 * kMaxCtas * 4);
     L.partials = o;    o += up256(static_cast<size_t>(2 * kMaxCtas) * 128 * L.acc_cols * 4);
     L.total = o;
     return true;
@@ -196,6 +198,7 @@ static int gemm_common(const moe_shape_t *shape, int mode, const void *act, cons
     if (ws_bytes < L.total) return MOE_ERR_WORKSPACE_TOO_SMALL;
     char *b = static_cast<char *>(ws);
     GemmArgs a;
+    a.chained = false;
     a.mode = mode;
     a.act = act;
     a.wgt = wgt;
@@ -275,19 +278,23 @@ int moe_fused_forward(const moe_shape_t *shape, const void *x, const float *logi
     void *h = b + L.h;
     float *y = reinterpret_cast<float *>(b + L.y);
 
-    cudaError_t e = cudaMemsetAsync(ctrl, 0, sizeof(Ctrl), sm);
+    // One memset clears the status, the align ticket and both GEMMs' tile
+    // counters.  Every later kernel is a programmatic dependent launch of the
+    // one before it, so there is no other non-kernel node in the sequence.
+    cudaError_t e = cudaMemsetAsync(ctrl, 0, L.counters + 4 * kMaxCtas * sizeof(int32_t) - L.ctrl, sm);
     if (e != cudaSuccess) return MOE_ERR_CUDA;
     e = launch_route(s, logits, ids, w, sm);
     if (e != cudaSuccess) return MOE_ERR_CUDA;
     g_launches += 1;
     e = launch_align(s, ids, counts, offsets, rows, inv, reinterpret_cast<int32_t *>(b + L.chunk_hist),
-                     reinterpret_cast<int32_t *>(b + L.chunk_base), ctrl, sm, &g_launches);
+                     reinterpret_cast<int32_t *>(b + L.chunk_base), ctrl, sm, &g_launches, true);
     if (e != cudaSuccess) return MOE_ERR_CUDA;
-    e = launch_gather(s, x, rows, offsets, a1_scale, xp, L.max_rows, sm);
+    e = launch_gather(s, x, rows, offsets, a1_scale, xp, L.max_rows, sm, true);
     if (e != cudaSuccess) return MOE_ERR_CUDA;
     g_launches += 1;
     const GemmPlan plan = plan_gemm(s);
     GemmArgs a;
+    a.chained = true;
     a.status = &ctrl->status;
     a.counters = reinterpret_cast<int32_t *>(b + L.counters);
     a.partials = reinterpret_cast<float *>(b + L.partials);
@@ -310,10 +317,11 @@ int moe_fused_forward(const moe_shape_t *shape, const void *x, const float *logi
     a.wscale = w2_scale;
     a.ascale = s.adtype == MOE_E4M3 ? a2_scale : 1.0f;
     a.out = y;
+    a.counters += 2 * kMaxCtas;
     e = launch_grouped_gemm(s, plan, a, sm, &g_launches, &host_err);
     if (host_err != MOE_OK) return host_err;
     if (e != cudaSuccess) return MOE_ERR_CUDA;
-    e = launch_combine(s, y, w, inv, offsets, out, sm);
+    e = launch_combine(s, y, w, inv, offsets, out, sm, true);
     if (e != cudaSuccess) return MOE_ERR_CUDA;
     g_launches += 1;
     return MOE_OK;

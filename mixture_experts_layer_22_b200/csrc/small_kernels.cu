@@ -47,6 +47,8 @@ __global__ void __launch_bounds__(256) route_topk_kernel(const float *__restrict
                                                          float routed_scale, int32_t *ids,
                                                          float *w)
 {
+    grid_dep_wait();
+    grid_dep_launch();
     const int lane = threadIdx.x & 31;
     const int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     if (t >= T) return;
@@ -133,6 +135,8 @@ __global__ void __launch_bounds__(1024) align_count_kernel(
     int32_t *chunk_hist, int32_t *chunk_base, int32_t *counts, int32_t *offsets,
     int32_t *sorted_rows, Ctrl *ctrl)
 {
+    grid_dep_wait();
+    grid_dep_launch();
     extern __shared__ int32_t sh[];
     __shared__ int s_last;
     const int Et = E + n_shared;
@@ -214,6 +218,8 @@ __global__ void __launch_bounds__(1024) align_scatter_kernel(const int32_t *__re
                                                              const int32_t *chunk_base,
                                                              int32_t *sorted_rows, int32_t *inv)
 {
+    grid_dep_wait();
+    grid_dep_launch();
     extern __shared__ int32_t wc[];   // [32 warps][Et]
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     for (int i = tid; i < 32 * Et; i += blockDim.x) wc[i] = 0;
@@ -254,6 +260,8 @@ __global__ void __launch_bounds__(1024) align_single_kernel(const int32_t *__res
                                                             int32_t *offsets, int32_t *sorted_rows,
                                                             int32_t *inv, Ctrl *ctrl)
 {
+    grid_dep_wait();
+    grid_dep_launch();
     extern __shared__ int32_t sm_al[];
     const int Et = E + n_shared;
     int32_t *hist = sm_al;                 // [Et]: counts, then segment starts
@@ -326,7 +334,7 @@ __global__ void __launch_bounds__(1024) align_single_kernel(const int32_t *__res
 
 cudaError_t launch_align(const moe_shape_t &s, const int32_t *ids, int32_t *counts,
                          int32_t *offsets, int32_t *sorted_rows, int32_t *inv, int32_t *chunk_hist,
-                         int32_t *chunk_base, Ctrl *ctrl, cudaStream_t st, int *launches)
+                         int32_t *chunk_base, Ctrl *ctrl, cudaStream_t st, int *launches, bool chained)
 {
     const int R = s.T * s.k, Et = s.E + s.n_shared;
     const int nb = (R + kAlignChunk - 1) / kAlignChunk;
@@ -339,19 +347,22 @@ cudaError_t launch_align(const moe_shape_t &s, const int32_t *ids, int32_t *coun
         attr_done = true;
     }
     if (nb == 1) {
-        align_single_kernel<<<1, kAlignChunk, 33 * Et * sizeof(int32_t), st>>>(ids, R, s.T, s.E, s.n_shared, s.pad,
-                                                                            counts, offsets, sorted_rows, inv, ctrl);
         *launches += 1;
-        return cudaGetLastError();
+        return launch_kernel(align_single_kernel, dim3(1), dim3(kAlignChunk), 33 * Et * sizeof(int32_t), st,
+                             chained, ids, R, s.T, s.E, s.n_shared, s.pad, counts, offsets, sorted_rows, inv,
+                             ctrl);
     }
-    cudaError_t err = cudaMemsetAsync(&ctrl->ticket, 0, sizeof(int32_t), st);
+    if (!chained) {
+        cudaError_t err = cudaMemsetAsync(&ctrl->ticket, 0, sizeof(int32_t), st);
+        if (err != cudaSuccess) return err;
+    }
+    cudaError_t err = launch_kernel(align_count_kernel, dim3(nb), dim3(kAlignChunk), Et * sizeof(int32_t), st,
+                                    chained, ids, R, s.T, s.E, s.n_shared, s.pad, chunk_hist, chunk_base,
+                                    counts, offsets, sorted_rows, ctrl);
     if (err != cudaSuccess) return err;
-    align_count_kernel<<<nb, kAlignChunk, Et * sizeof(int32_t), st>>>(
-        ids, R, s.T, s.E, s.n_shared, s.pad, chunk_hist, chunk_base, counts, offsets, sorted_rows, ctrl);
-    align_scatter_kernel<<<nb, kAlignChunk, 32 * Et * sizeof(int32_t), st>>>(ids, R, s.E, Et, chunk_base,
-                                                                             sorted_rows, inv);
     *launches += 2;
-    return cudaGetLastError();
+    return launch_kernel(align_scatter_kernel, dim3(nb), dim3(kAlignChunk), 32 * Et * sizeof(int32_t), st,
+                         chained, ids, R, s.E, Et, static_cast<const int32_t *>(chunk_base), sorted_rows, inv);
 }
 
 // ------------------------------------------------------------------ gather
@@ -362,6 +373,8 @@ __global__ void __launch_bounds__(256) gather_kernel(const uint4 *__restrict__ x
                                                      const int32_t *__restrict__ offsets, int Et,
                                                      int T, int k, int H, float a1, void *xp)
 {
+    grid_dep_wait();
+    grid_dep_launch();
     const int lane = threadIdx.x & 31;
     const int nvec = H / 8;                       // 8 bf16 per 16 bytes
     const int nchunk = (nvec + 31) / 32;          // 512-byte chunks per row
@@ -402,20 +415,16 @@ __global__ void __launch_bounds__(256) gather_kernel(const uint4 *__restrict__ x
 
 cudaError_t launch_gather(const moe_shape_t &s, const void *x, const int32_t *sorted_rows,
                           const int32_t *offsets, float a1, void *xp, int64_t max_rows,
-                          cudaStream_t st)
+                          cudaStream_t st, bool chained)
 {
     const int Et = s.E + s.n_shared;
     const int64_t warps = max_rows * ((s.H / 8 + 31) / 32);
     int blocks = static_cast<int>((warps + 7) / 8);
     if (blocks > 148 * 16) blocks = 148 * 16;
     if (blocks < 1) blocks = 1;
-    if (s.adtype == MOE_E4M3)
-        gather_kernel<true><<<blocks, 256, 0, st>>>(static_cast<const uint4 *>(x), sorted_rows, offsets,
-                                                    Et, s.T, s.k, s.H, a1, xp);
-    else
-        gather_kernel<false><<<blocks, 256, 0, st>>>(static_cast<const uint4 *>(x), sorted_rows,
-                                                     offsets, Et, s.T, s.k, s.H, a1, xp);
-    return cudaGetLastError();
+    return launch_kernel(s.adtype == MOE_E4M3 ? gather_kernel<true> : gather_kernel<false>, dim3(blocks),
+                         dim3(256), 0, st, chained, static_cast<const uint4 *>(x), sorted_rows, offsets, Et,
+                         s.T, s.k, s.H, a1, xp);
 }
 
 // ------------------------------------------------------------------ combine
@@ -427,6 +436,8 @@ __global__ void __launch_bounds__(256) combine_kernel(const float4 *__restrict__
                                                       const int32_t *__restrict__ offsets, int H,
                                                       int k, int E, int n_shared, uint2 *out)
 {
+    grid_dep_wait();
+    grid_dep_launch();
     const int t = blockIdx.x;
     const int n4 = H / 4;
     __shared__ int s_slot[kMaxTopK + 1];
@@ -466,12 +477,12 @@ __global__ void __launch_bounds__(256) combine_kernel(const float4 *__restrict__
 }
 
 cudaError_t launch_combine(const moe_shape_t &s, const float *y, const float *w,
-                           const int32_t *inv, const int32_t *offsets, void *out, cudaStream_t st)
+                           const int32_t *inv, const int32_t *offsets, void *out, cudaStream_t st,
+                           bool chained)
 {
     const dim3 grid(s.T, (s.H / 4 + 255) / 256);
-    combine_kernel<<<grid, 256, 0, st>>>(reinterpret_cast<const float4 *>(y), w, inv, offsets, s.H,
-                                         s.k, s.E, s.n_shared, static_cast<uint2 *>(out));
-    return cudaGetLastError();
+    return launch_kernel(combine_kernel, grid, dim3(256), 0, st, chained, reinterpret_cast<const float4 *>(y),
+                         w, inv, offsets, s.H, s.k, s.E, s.n_shared, static_cast<uint2 *>(out));
 }
 
 }  // namespace moe
