@@ -188,6 +188,12 @@ int moe_gather(const moe_shape_t *shape, const void *x, const int32_t *sorted_ro
  *   fp32 accumulation in tensor memory; every weight byte of an expert is
  *   read once per call in the Swap-AB variant when the expert has at most
  *   256 rows.
+ *   E4M3 weights with bf16 activations (this call and step 5): the
+ *   activation rows are first split, in the workspace, into two E4M3 planes
+ *   with one power-of-two scale s per row, v = s * (hi + lo), and the GEMM
+ *   runs on the E4M3 tensor path.  The split is exact except for elements
+ *   below about 2^-11 of their row's largest magnitude, which are off by at
+ *   most 2^-10 s.
  */
 int moe_grouped_gemm_swiglu(const moe_shape_t *shape, const void *xp, const void *w13,
                             const float *w13_scale, float a1_scale, float a2_scale,

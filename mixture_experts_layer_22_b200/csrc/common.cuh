@@ -63,6 +63,7 @@ struct WsLayout {
     size_t total;
     int64_t max_rows;
     int n_chunks;
+    size_t planes, rowscale;   // E4M3 weights + bf16 activations only (else 0 bytes)
     int acc_cols;         // accumulator columns of the widest GEMM tile
 };
 
@@ -93,6 +94,13 @@ cudaError_t launch_combine(const moe_shape_t &s, const float *y, const float *w,
                            const int32_t *inv, const int32_t *offsets, void *out,
                            cudaStream_t st, bool chained = false);
 
+// Split bf16 rows [offsets[E+n_shared], K] of `src` into E4M3 planes hi
+// (rows 0..) and lo (rows max_rows..) of `planes` with v = scale[row] *
+// (hi + lo); see small_kernels.cu.
+cudaError_t launch_split_hilo(const moe_shape_t &s, const void *src, int K, const int32_t *offsets,
+                              void *planes, float *scale, int64_t max_rows, cudaStream_t st,
+                              bool chained);
+
 struct GemmArgs {
     int mode;                 // 0: gate/up + SwiGLU, 1: down projection
     const void *act;          // xp or h
@@ -106,6 +114,8 @@ struct GemmArgs {
     float *partials;
     int64_t max_rows;
     bool chained;             // PDL launch; counters already zero
+    void *planes;             // E4M3 weights + bf16 activations: hi/lo activation planes
+    float *rowscale;          //   [2 * max_rows, K] E4M3 and the scale of each row
 };
 cudaError_t launch_grouped_gemm(const moe_shape_t &s, const GemmPlan &p, const GemmArgs &a,
                                 cudaStream_t st, int *launches, int *host_err);

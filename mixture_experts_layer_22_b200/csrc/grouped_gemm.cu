@@ -55,6 +55,8 @@ struct GemmParams {
     int32_t *status;
     int32_t *counters;
     float *partials;
+    const float *rowscale;   // kHiLo: scale of each permuted activation row
+    int lo_rows;             // kHiLo: row offset of the lo plane in the activation map
     int pdl;          // launched as a programmatic dependent: prefetch the first weight
                       // stages into L2 before waiting for the previous kernel
     int stream_k;     // 0: whole tiles only.  Otherwise whole tiles for all but the
@@ -66,7 +68,7 @@ struct GemmParams {
                       // 2 (tensor-bound prefill): rounds >= 90% full on average.
 };
 
-template <int kMode, bool kSwap, bool kFp8, int kBN, bool kW8 = false>
+template <int kMode, bool kSwap, bool kFp8, int kBN, bool kHiLo = false>
 struct Cfg {
     // K bytes per operand row and stage (128: the 128-byte swizzle; 64-byte
     // rows with the 64-byte swizzle are supported by the loads and
@@ -74,38 +76,30 @@ struct Cfg {
     static constexpr int kRowBytes = 128;
     static constexpr int kMmaPerStage = kRowBytes / 32;     // 32 bytes of K per MMA
     static constexpr int kStageA = 128 * kRowBytes;          // 128 rows
-    static constexpr int kStageB = kBN * kRowBytes;
+    // kHiLo (E4M3 weights, bf16 activations): each token row arrives as two
+    // E4M3 planes (hi, lo), stacked in N: rows [0, n) hi, [n, 2n) lo
+    static constexpr int kPlanes = kHiLo ? 2 : 1;
+    static constexpr int kStageB = kPlanes * kBN * kRowBytes;
     static constexpr int kStage = kStageA + kStageB;
     static constexpr int kDynBudget = 205 * 1024;
     static constexpr int kStagesRaw = kDynBudget / kStage;
-    static constexpr int kStagesFull = kStagesRaw > 12 ? 12 : kStagesRaw;
-    // E4M3 weights with bf16 activations (kW8): one smem stage holds a raw
-    // E4M3 weight tile (128 rows x 128 codes) and the bf16 activation rows of
-    // both K halves; the converted bf16 weight slabs (K = 64, 32 columns) go
-    // to tensor memory, from where the MMA reads its A operand.
-    static constexpr int kStageW8 = kStageA + 2 * kStageB;
-    static constexpr int kStagesW8Fit = kDynBudget / kStageW8;
-    static constexpr int kStagesW8 = kStagesW8Fit > 10 ? 10 : kStagesW8Fit;
-    static constexpr int kStages = kW8 ? kStagesW8 : kStagesFull;
-    static constexpr int kDynSmem = (kW8 ? kStagesW8 * kStageW8 : kStagesFull * kStage) + 1024;
+    static constexpr int kStages = kStagesRaw > 12 ? 12 : kStagesRaw;
+    static constexpr int kDynSmem = kStages * kStage + 1024;
     // epilogue warps 2 .. 2+kEpiWarps-1; the normal order uses two per
     // tensor-memory lane quarter, each taking half of the tile's columns
     static constexpr int kEpiWarps = kSwap ? 4 : 8;
     static constexpr int kEpiThreads = 32 * kEpiWarps;
-    static constexpr int kThreads = kW8 ? 480 : 64 + kEpiThreads;   // kW8: + 8 converters + a 2nd MMA warp
-    static constexpr int kAccCols = kSwap ? kBN : 256;      // fp32 columns per accumulator
-    // kW8: each accumulator buffer has two halves (one per MMA warp / K half)
-    static constexpr int kAccSplit = kW8 ? 2 : 1;
-    static constexpr int kTmemCols = kW8 ? 512 : ((2 * kAccCols) <= 32 ? 32 : 2 * kAccCols);
-    static constexpr int kAColBase = 2 * kAccSplit * kAccCols;       // first TMEM column of the A slabs
-    static constexpr int kAStages = 8;                               // A slabs of 32 columns (4 pairs)
+    static constexpr int kThreads = 64 + kEpiThreads;
+    static constexpr int kAccCols = kSwap ? kPlanes * kBN : 256;   // fp32 columns per accumulator
+    static constexpr int kTmemCols = (2 * kAccCols) <= 32 ? 32 : 2 * kAccCols;
     static constexpr int kRowsTile = kSwap ? kBN : 128;     // token rows per tile
     static constexpr int kFeatTile = kMode == 0 ? (kSwap ? 64 : 128) : (kSwap ? 128 : 256);
-    static constexpr int kKStage = (kFp8 || kW8) ? kRowBytes : kRowBytes / 2;   // K elements per work step
+    static constexpr int kKStage = kFp8 ? kRowBytes : kRowBytes / 2;   // K elements per work step
     static constexpr uint32_t kFmt = kFp8 ? 0u : 1u;
-    static_assert(kW8 ? kStagesW8 >= 4 : kStagesFull >= 2, "smem ring too small");
-    static_assert(!kW8 || (kSwap && !kFp8 && kBN <= 64), "E4M3-weight/bf16-activation path: Swap-AB, BN <= 64");
-    static_assert(!kW8 || kAColBase + kAStages * 32 <= 512, "tensor memory for the A slabs");
+    // h leaves GEMM1 as E4M3 only on the all-E4M3 path
+    static constexpr bool kOutE4M3 = kFp8 && !kHiLo;
+    static_assert(kStages >= 2, "smem ring too small");
+    static_assert(!kHiLo || (kSwap && kFp8 && kBN <= 128), "hi/lo planes: Swap-AB on the E4M3 tensor path");
     static_assert(kTmemCols <= 512, "tensor memory");
 };
 
@@ -227,40 +221,6 @@ __device__ __forceinline__ uint32_t e4m3_code(float v)
     return static_cast<uint32_t>(__nv_cvt_float_to_fp8(v, __NV_SATFINITE, __NV_E4M3)) & 0xFFu;
 }
 
-// Four E4M3 codes (one 32-bit word, first code in the low byte) -> four bf16
-// values (two bf16x2 words, K order), exactly.  Each code's bits are placed
-// so that the bf16 exponent field holds the E4M3 exponent field unchanged
-// (s 0000 eeee mmm 0000), which is the bf16 number w * 2^-120 for normal AND
-// subnormal codes; one bf16 multiply by 2^120 then gives w exactly.  Codes
-// 0x7F/0xFF (NaN) are not valid weights.
-__device__ __forceinline__ void e4m3x4_to_bf16(uint32_t w, uint32_t &lo, uint32_t &hi)
-{
-    const uint32_t two120 = 0x7B807B80u;   // bf16x2 {2^120, 2^120}
-    uint32_t t0 = __byte_perm(w, 0u, 0x1404u);   // {b1 << 8, b0 << 8}
-    uint32_t t1 = __byte_perm(w, 0u, 0x3424u);   // {b3 << 8, b2 << 8}
-    t0 >>= 4;                                    // {b1 << 4, b0 << 4}: sign at bit 11
-    t1 >>= 4;
-    t0 += 15u * (t0 & 0x08000800u);              // move the sign from bit 11 to bit 15
-    t1 += 15u * (t1 & 0x08000800u);
-    asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(lo) : "r"(t0), "r"(two120));
-    asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(hi) : "r"(t1), "r"(two120));
-}
-
-// 64 E4M3 codes (four 16-byte chunks of one swizzled 128-byte row) -> 64
-// bf16 values packed two per 32-bit word, K order.
-__device__ __forceinline__ void e4m3x64_to_bf16(const uint8_t *row, int r, int half, uint32_t (&o)[32])
-{
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-        const int c = 4 * half + q;
-        const uint4 v = *reinterpret_cast<const uint4 *>(row + ((c ^ (r & 7)) << 4));
-        e4m3x4_to_bf16(v.x, o[q * 8 + 0], o[q * 8 + 1]);
-        e4m3x4_to_bf16(v.y, o[q * 8 + 2], o[q * 8 + 3]);
-        e4m3x4_to_bf16(v.z, o[q * 8 + 4], o[q * 8 + 5]);
-        e4m3x4_to_bf16(v.w, o[q * 8 + 6], o[q * 8 + 7]);
-    }
-}
-
 // Wait (bounded, ignoring the abort flag) for the last `issued` fills of a
 // ring whose next stage/phase is (stage, phase): lets in-flight TMA copies
 // land before an aborting CTA exits.
@@ -274,17 +234,17 @@ __device__ __forceinline__ void drain_ring(uint64_t *full, int nstages, int stag
     }
 }
 
-template <int kMode, bool kSwap, bool kFp8, int kBN, bool kW8 = false>
-__global__ void __launch_bounds__(Cfg<kMode, kSwap, kFp8, kBN, kW8>::kThreads, 1)
+template <int kMode, bool kSwap, bool kFp8, int kBN, bool kHiLo = false>
+__global__ void __launch_bounds__(Cfg<kMode, kSwap, kFp8, kBN, kHiLo>::kThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tm_w,
                         const __grid_constant__ CUtensorMap tm_x, GemmParams p)
 {
-    using C = Cfg<kMode, kSwap, kFp8, kBN, kW8>;
+    using C = Cfg<kMode, kSwap, kFp8, kBN, kHiLo>;
     extern __shared__ uint8_t dyn_smem[];
     __shared__ int s_off[kMaxExpertsTotal + 1];
     __shared__ int s_prefix[kMaxExpertsTotal + 1];
     __shared__ __align__(8) uint64_t s_full[C::kStages], s_empty[C::kStages];
-    __shared__ __align__(8) uint64_t s_tfull[2], s_tempty[2], s_drain, s_drain2;
+    __shared__ __align__(8) uint64_t s_tfull[2], s_tempty[2], s_drain;
     __shared__ uint32_t s_tmem_base;
     __shared__ volatile int s_abort;
     __shared__ int s_is_last;
@@ -294,8 +254,6 @@ __global__ void __launch_bounds__(Cfg<kMode, kSwap, kFp8, kBN, kW8>::kThreads, 1
     // bank conflicts) so that the output is written as whole row segments
     constexpr int kStagePitch = 80;
     __shared__ __align__(16) uint8_t s_out_stage[kSwap ? 16 : C::kEpiWarps * 32 * kStagePitch];
-    constexpr int kAN = kW8 ? C::kAStages : 1;
-    __shared__ __align__(8) uint64_t s_a_full[kAN];
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int Et = p.E_tot;
@@ -307,20 +265,13 @@ __global__ void __launch_bounds__(Cfg<kMode, kSwap, kFp8, kBN, kW8>::kThreads, 1
         s_abort = 0;
         for (int i = 0; i < C::kStages; ++i) {
             mbar_init(smem_u32(&s_full[i]), 1);
-            // kW8: the stage is free once its 4 converter warps have read the
-            // raw tile and both MMA warps have read the activations
-            mbar_init(smem_u32(&s_empty[i]), kW8 ? 6 : 1);
+            mbar_init(smem_u32(&s_empty[i]), 1);
         }
         for (int i = 0; i < 2; ++i) {
-            mbar_init(smem_u32(&s_tfull[i]), kW8 ? 2 : 1);
+            mbar_init(smem_u32(&s_tfull[i]), 1);
             mbar_init(smem_u32(&s_tempty[i]), C::kEpiWarps);
         }
         mbar_init(smem_u32(&s_drain), 1);
-        mbar_init(smem_u32(&s_drain2), 1);
-        if (kW8) {
-            for (int i = 0; i < kAN; ++i)                      // one barrier per slab pair
-                mbar_init(smem_u32(&s_a_full[i]), 4);         // the four warps of a converter group
-        }
         fence_mbar_init();
         prefetch_tmap(&tm_w);
         prefetch_tmap(&tm_x);
@@ -411,155 +362,7 @@ __global__ void __launch_bounds__(Cfg<kMode, kSwap, kFp8, kBN, kW8>::kThreads, 1
     grid_dep_launch();
 
 
-    if (kW8 && warp == 0) {
-        // ================= TMA producer (E4M3 weights, bf16 activations) ====
-        if (lane == 0) {
-            const uint64_t pol_w = policy_evict_first();
-            const uint64_t pol_x = policy_evict_last();
-            int stage = 0, in_flight = 0;
-            uint32_t phase = 0;
-            ItemIter I;
-            iter_init(I, S, blockIdx.x);
-            Item it;
-            bool ok = true;
-            while (ok && iter_next<C::kRowsTile>(I, S, s_prefix, s_off, Et, n_ft, it)) {
-                const int row0 = s_off[it.e] + it.rt * C::kRowsTile;
-                const int rows = min(C::kRowsTile, s_off[it.e + 1] - row0);
-                const int wbase = it.e * p.w_rows;
-                for (int kk = it.kb; kk < it.ke; ++kk) {
-                    if (!mbar_wait(smem_u32(&s_empty[stage]), phase ^ 1u, &s_abort)) {
-                        ok = false;
-                        break;
-                    }
-                    const uint32_t fb = smem_u32(&s_full[stage]);
-                    mbar_arrive_expect_tx(fb, C::kStageA + 2 * rows * 128);
-                    const uint32_t sa = smem_u32(tiles + stage * C::kStageW8);
-                    const int kx8 = kk * 128;                      // E4M3 elements
-                    if (kMode == 0) {
-                        tma_load_2d(sa, &tm_w, fb, kx8, wbase + it.ft * 64, pol_w);
-                        tma_load_2d(sa + 64 * 128, &tm_w, fb, kx8, wbase + p.n_feat + it.ft * 64, pol_w);
-                    } else {
-                        tma_load_2d(sa, &tm_w, fb, kx8, wbase + it.ft * 128, pol_w);
-                    }
-                    for (int hh = 0; hh < 2; ++hh)
-                        for (int rr = 0; rr < rows; rr += 16)
-                            tma_load_2d(sa + C::kStageA + hh * C::kStageB + rr * 128, &tm_x, fb,
-                                        kk * 128 + hh * 64, row0 + rr, pol_x);
-                    ++in_flight;
-                    if (++stage == C::kStages) {
-                        stage = 0;
-                        phase ^= 1u;
-                    }
-                }
-            }
-            if (!ok) drain_ring(s_full, C::kStages, stage, phase, in_flight);
-        }
-    } else if (kW8 && warp >= 6 && warp <= 13) {
-        // ================= E4M3 -> bf16 converters (warps 6..13) ============
-        // Two groups of four warps take alternate stages (group g: stages
-        // j = g, g+2, ...), so two stages are converted at once.  Warp w
-        // covers the 32 weight rows of its tensor-memory lane quarter (w % 4):
-        // thread = one row, both K halves (2 x 64 codes -> 2 x 32 packed
-        // columns), stored into slab pair j % 4 with tcgen05.st.  Slab pair
-        // j % 4 is free once stage j-4 has been released (its release needs
-        // both MMA warps' commits, i.e. its MMAs have completed).
-        const int group = (warp - 6) >> 2;
-        const int q = warp & 3;
-        const int r = q * 32 + lane;
-        const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
-        int stage = 0, j = 0;
-        uint32_t phase = 0;
-        ItemIter I;
-        iter_init(I, S, blockIdx.x);
-        Item it;
-        bool ok = true;
-        while (ok && iter_next<C::kRowsTile>(I, S, s_prefix, s_off, Et, n_ft, it)) {
-            for (int kk = it.kb; kk < it.ke; ++kk, ++j) {
-                if ((j & 1) == group) {
-                    const int pr = j & 3;
-                    bool got = mbar_wait(smem_u32(&s_full[stage]), phase, &s_abort);
-                    if (got && j >= 4) {
-                        const int jp = j - 4;
-                        got = mbar_wait(smem_u32(&s_empty[jp % C::kStages]),
-                                        static_cast<uint32_t>(jp / C::kStages) & 1u, &s_abort);
-                    }
-                    if (!got) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
-                    const uint8_t *row = tiles + stage * C::kStageW8 + r * 128;
-                    uint32_t o[32];
-                    e4m3x64_to_bf16(row, r, 0, o);
-                    tmem_st32(tmem_base + lane_base + C::kAColBase + (2 * pr) * 32, o);
-                    e4m3x64_to_bf16(row, r, 1, o);
-                    tmem_st32(tmem_base + lane_base + C::kAColBase + (2 * pr + 1) * 32, o);
-                    tmem_wait_st();
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) {
-                        mbar_arrive(smem_u32(&s_a_full[pr]));
-                        mbar_arrive(smem_u32(&s_empty[stage]));
-                    }
-                }
-                if (++stage == C::kStages) {
-                    stage = 0;
-                    phase ^= 1u;
-                }
-            }
-        }
-    } else if (kW8 && (warp == 1 || warp == 14)) {
-        // ================= MMA issuers (A = bf16 slabs in TMEM, B = smem) ===
-        // Warp 1 issues the K half 0 MMAs of every stage, warp 14 those of
-        // K half 1, each into its own half of the accumulator buffer; the
-        // epilogue adds the two halves.
-        if (lane == 0) {
-            const int hh = warp == 1 ? 0 : 1;
-            int stage = 0, acc = 0, j = 0;
-            uint32_t acc_phase = 0;
-            ItemIter I;
-            iter_init(I, S, blockIdx.x);
-            Item it;
-            bool ok = true;
-            while (ok && iter_next<C::kRowsTile>(I, S, s_prefix, s_off, Et, n_ft, it)) {
-                if (!mbar_wait(smem_u32(&s_tempty[acc]), acc_phase ^ 1u, &s_abort)) break;
-                tc_fence_after();
-                const uint32_t d = tmem_base + (acc * 2 + hh) * C::kAccCols;
-                const int seg = s_off[it.e + 1] - s_off[it.e];
-                const int n = min(C::kRowsTile, seg - it.rt * C::kRowsTile);
-                const uint32_t idesc = idesc_make(1u, 128, n);
-                for (int kk = it.kb; kk < it.ke; ++kk, ++j) {
-                    const int pr = j & 3;
-                    // the converters arrive on a_full only after observing the
-                    // stage's full barrier, so the activation rows have landed too
-                    if (!mbar_wait(smem_u32(&s_a_full[pr]), static_cast<uint32_t>(j >> 2) & 1u, &s_abort)) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
-                    const uint32_t ta = tmem_base + C::kAColBase + (2 * pr + hh) * 32;
-                    const uint32_t sb = smem_u32(tiles + stage * C::kStageW8 + C::kStageA + hh * C::kStageB);
-                    const uint64_t bd0 = sdesc_k_sw128(sb);
-#pragma unroll
-                    for (int s4 = 0; s4 < 4; ++s4)
-                        mma_bf16_tmem_a(d, ta + s4 * 8, bd0 + static_cast<uint64_t>(s4 * 2), idesc,
-                                        (kk > it.kb || s4 > 0) ? 1u : 0u);
-                    mma_commit(smem_u32(&s_empty[stage]));
-                    if (++stage == C::kStages) stage = 0;
-                }
-                if (!ok) break;
-                mma_commit(smem_u32(&s_tfull[acc]));
-                if (++acc == 2) {
-                    acc = 0;
-                    acc_phase ^= 1u;
-                }
-            }
-            uint64_t *dr = warp == 1 ? &s_drain : &s_drain2;
-            mma_commit(smem_u32(dr));
-            volatile int no_abort = 0;
-            mbar_wait(smem_u32(dr), 0, &no_abort);
-        }
-    } else if (!kW8 && warp == 0) {
+    if (warp == 0) {
         // ================= TMA producer =================
         if (lane == 0) {
             // Swap-AB (few token rows per expert) streams every weight byte
@@ -585,8 +388,9 @@ __global__ void __launch_bounds__(Cfg<kMode, kSwap, kFp8, kBN, kW8>::kThreads, 1
                         break;
                     }
                     const uint32_t fb = smem_u32(&s_full[stage]);
-                    // Swap-AB: only the tile's own token rows (16-row boxes)
-                    mbar_arrive_expect_tx(fb, kSwap ? C::kStageA + rows * C::kRowBytes : C::kStage);
+                    // Swap-AB: only the tile's own token rows (16-row boxes), of
+                    // both planes for kHiLo
+                    mbar_arrive_expect_tx(fb, kSwap ? C::kStageA + C::kPlanes * rows * C::kRowBytes : C::kStage);
                     const uint32_t sa = smem_u32(tiles + stage * C::kStage);
                     const uint32_t sb = sa + C::kStageA;
                     const int kx = kk * C::kKStage;
@@ -599,6 +403,9 @@ __global__ void __launch_bounds__(Cfg<kMode, kSwap, kFp8, kBN, kW8>::kThreads, 1
                         }
                         for (int rr = 0; rr < rows; rr += 16)
                             tma_load_2d(sb + rr * C::kRowBytes, &tm_x, fb, kx, row0 + rr, pol_x);
+                        if (kHiLo)
+                            for (int rr = 0; rr < rows; rr += 16)
+                                tma_load_2d(sb + (rows + rr) * C::kRowBytes, &tm_x, fb, kx, p.lo_rows + row0 + rr, pol_x);
                     } else {
                         tma_load_2d(sa, &tm_x, fb, kx, row0, pol_x);
                         if (kMode == 0) {
@@ -617,7 +424,7 @@ __global__ void __launch_bounds__(Cfg<kMode, kSwap, kFp8, kBN, kW8>::kThreads, 1
             }
             if (!ok) drain_ring(s_full, C::kStages, stage, phase, in_flight);   // let issued copies land
         }
-    } else if (!kW8 && warp == 1) {
+    } else if (warp == 1) {
         // ================= MMA issuer =================
         if (lane == 0) {
             int stage = 0;
@@ -635,7 +442,7 @@ __global__ void __launch_bounds__(Cfg<kMode, kSwap, kFp8, kBN, kW8>::kThreads, 1
                 int n = 256;
                 if (kSwap) {
                     const int seg = s_off[it.e + 1] - s_off[it.e];
-                    n = min(C::kRowsTile, seg - it.rt * C::kRowsTile);
+                    n = C::kPlanes * min(C::kRowsTile, seg - it.rt * C::kRowsTile);
                 }
                 const uint32_t idesc = idesc_make(C::kFmt, 128, n);
                 for (int kk = it.kb; kk < it.ke; ++kk) {
@@ -691,14 +498,17 @@ __global__ void __launch_bounds__(Cfg<kMode, kSwap, kFp8, kBN, kW8>::kThreads, 1
             const int seg = s_off[it.e + 1] - s_off[it.e];
             const int row0 = s_off[it.e] + it.rt * C::kRowsTile;
             const int rows = min(C::kRowsTile, seg - it.rt * C::kRowsTile);
-            const float sc = p.ascale * (p.wscale ? __ldg(&p.wscale[it.e]) : 1.0f);
-            const uint32_t tacc = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * C::kAccSplit * C::kAccCols;
-            // 16 accumulator columns starting at c0 (kW8: sum of the two halves)
+            // output scale of the tile; kHiLo: times the activation row's own
+            // scale (column j of a Swap-AB tile is permuted row row0 + j)
+            const float sc = (kHiLo ? 1.0f : p.ascale) * (p.wscale ? __ldg(&p.wscale[it.e]) : 1.0f);
+            auto col_sc = [&](int j) -> float { return kHiLo ? sc * __ldg(&p.rowscale[row0 + j]) : sc; };
+            const uint32_t tacc = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * C::kAccCols;
+            // 16 accumulator columns starting at c0 (kHiLo: hi plane + lo plane)
             auto ld_acc16 = [&](int c0, uint32_t (&v)[16]) {
                 tmem_ld16(tacc + c0, v);
-                if constexpr (kW8) {
+                if constexpr (kHiLo) {
                     uint32_t w2[16];
-                    tmem_ld16(tacc + C::kAccCols + c0, w2);
+                    tmem_ld16(tacc + rows + c0, w2);
                     tmem_wait_ld();
 #pragma unroll
                     for (int i2 = 0; i2 < 16; ++i2) v[i2] = __float_as_uint(__uint_as_float(v[i2]) + __uint_as_float(w2[i2]));
@@ -720,11 +530,12 @@ __global__ void __launch_bounds__(Cfg<kMode, kSwap, kFp8, kBN, kW8>::kThreads, 1
                         if (q < 2) {
 #pragma unroll
                             for (int j = 0; j < 16; ++j) {
-                                const float g = __uint_as_float(v[j]) * sc;
-                                const float u = s_xchg[j * 64 + r] * sc;
+                                const float scj = col_sc(c0 + j);
+                                const float g = __uint_as_float(v[j]) * scj;
+                                const float u = s_xchg[j * 64 + r] * scj;
                                 const float hv = silu_mul(g, u);
                                 const size_t o = static_cast<size_t>(row0 + c0 + j) * p.out_ld + f0 + r;
-                                if (kFp8)
+                                if (C::kOutE4M3)
                                     static_cast<uint8_t *>(p.out)[o] = static_cast<uint8_t>(e4m3_code(hv / p.qscale));
                                 else
                                     static_cast<__nv_bfloat16 *>(p.out)[o] = __float2bfloat16_rn(hv);
@@ -741,13 +552,13 @@ __global__ void __launch_bounds__(Cfg<kMode, kSwap, kFp8, kBN, kW8>::kThreads, 1
 #pragma unroll
                         for (int j = 0; j < 16; ++j)
                             static_cast<float *>(p.out)[static_cast<size_t>(row0 + c0 + j) * p.out_ld + h0 + r] =
-                                __uint_as_float(v[j]) * sc;
+                                __uint_as_float(v[j]) * col_sc(c0 + j);
                     }
                 } else if (kMode == 0) {
                     // 32 features per chunk: h row segment of 64 (bf16) or 32 (E4M3) bytes
                     const int f0 = it.ft * 128;
                     uint8_t *stg = s_out_stage + (warp - 2) * 32 * kStagePitch;
-                    const float inv_q = kFp8 ? 1.0f / p.qscale : 1.0f;
+                    const float inv_q = C::kOutE4M3 ? 1.0f / p.qscale : 1.0f;
                     for (int c0 = ch * (128 / kNch); c0 < (ch + 1) * (128 / kNch); c0 += 32) {
                         uint32_t g[16], u[16], g2[16], u2[16];
                         tmem_ld16(tacc + c0, g);
@@ -762,7 +573,7 @@ __global__ void __launch_bounds__(Cfg<kMode, kSwap, kFp8, kBN, kW8>::kThreads, 1
                             hv[16 + j] = silu_mul(__uint_as_float(g2[j]) * sc, __uint_as_float(u2[j]) * sc);
                         }
                         uint4 *wr = reinterpret_cast<uint4 *>(stg + lane * kStagePitch);
-                        if (kFp8) {
+                        if (C::kOutE4M3) {
 #pragma unroll
                             for (int j = 0; j < 2; ++j) {
                                 uint32_t w4[4];
@@ -781,9 +592,9 @@ __global__ void __launch_bounds__(Cfg<kMode, kSwap, kFp8, kBN, kW8>::kThreads, 1
                                                    pack_bf16x2(hv[8 * j + 4], hv[8 * j + 5]), pack_bf16x2(hv[8 * j + 6], hv[8 * j + 7]));
                         }
                         __syncwarp();
-                        constexpr int kSegLanes = kFp8 ? 2 : 4;          // 16-byte pieces per row segment
+                        constexpr int kSegLanes = C::kOutE4M3 ? 2 : 4;          // 16-byte pieces per row segment
                         constexpr int kRowsPerPass = 32 / kSegLanes;
-                        const size_t esz = kFp8 ? 1 : 2;
+                        const size_t esz = C::kOutE4M3 ? 1 : 2;
 #pragma unroll
                         for (int ps = 0; ps < kSegLanes; ++ps) {
                             const int rl = ps * kRowsPerPass + lane / kSegLanes;
@@ -871,9 +682,10 @@ __global__ void __launch_bounds__(Cfg<kMode, kSwap, kFp8, kBN, kW8>::kThreads, 1
                                 g += __ldcg(&ps[j * 128 + rr]);
                                 u += __ldcg(&ps[j * 128 + 64 + rr]);
                             }
-                            const float hv = silu_mul(g * sc, u * sc);
+                            const float scj = col_sc(j);
+                            const float hv = silu_mul(g * scj, u * scj);
                             const size_t o = static_cast<size_t>(row0 + j) * p.out_ld + f0 + rr;
-                            if (kFp8) static_cast<uint8_t *>(p.out)[o] = static_cast<uint8_t>(e4m3_code(hv / p.qscale));
+                            if (C::kOutE4M3) static_cast<uint8_t *>(p.out)[o] = static_cast<uint8_t>(e4m3_code(hv / p.qscale));
                             else static_cast<__nv_bfloat16 *>(p.out)[o] = __float2bfloat16_rn(hv);
                         }
                     } else if (kSwap) {
@@ -881,7 +693,7 @@ __global__ void __launch_bounds__(Cfg<kMode, kSwap, kFp8, kBN, kW8>::kThreads, 1
                         for (int j = 0; j < ncols; ++j) {
                             float a = 0.f;
                             for (int c = c_first; c <= c_last; ++c) a += __ldcg(&slot_of(c)[j * 128 + etid]);
-                            static_cast<float *>(p.out)[static_cast<size_t>(row0 + j) * p.out_ld + h0 + etid] = a * sc;
+                            static_cast<float *>(p.out)[static_cast<size_t>(row0 + j) * p.out_ld + h0 + etid] = a * col_sc(j);
                         }
                     } else if (kMode == 0) {
                         const int f0 = it.ft * 128;
@@ -896,7 +708,7 @@ __global__ void __launch_bounds__(Cfg<kMode, kSwap, kFp8, kBN, kW8>::kThreads, 1
                                 }
                                 const float hv = silu_mul(g * sc, u * sc);
                                 const size_t o = static_cast<size_t>(row0 + rr) * p.out_ld + f0 + j;
-                                if (kFp8) static_cast<uint8_t *>(p.out)[o] = static_cast<uint8_t>(e4m3_code(hv / p.qscale));
+                                if (C::kOutE4M3) static_cast<uint8_t *>(p.out)[o] = static_cast<uint8_t>(e4m3_code(hv / p.qscale));
                                 else static_cast<__nv_bfloat16 *>(p.out)[o] = __float2bfloat16_rn(hv);
                             }
                     } else {
@@ -982,18 +794,18 @@ static int sm_count()
     return n;
 }
 
-template <int kMode, bool kSwap, bool kFp8, int kBN, bool kW8 = false>
+template <int kMode, bool kSwap, bool kFp8, int kBN, bool kHiLo = false>
 static cudaError_t run_gemm(const moe_shape_t &s, const GemmArgs &a, cudaStream_t st, int *host_err)
 {
-    using Cf = Cfg<kMode, kSwap, kFp8, kBN, kW8>;
-    auto kern = grouped_gemm_kernel<kMode, kSwap, kFp8, kBN, kW8>;
+    using Cf = Cfg<kMode, kSwap, kFp8, kBN, kHiLo>;
+    auto kern = grouped_gemm_kernel<kMode, kSwap, kFp8, kBN, kHiLo>;
     static std::once_flag once;
     std::call_once(once, [&] {
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cf::kDynSmem);
     });
     const int Et = s.E + s.n_shared;
     const bool u8 = kFp8;              // activations are E4M3 codes
-    const bool u8w = kFp8 || kW8;      // weights are E4M3 codes
+    const bool u8w = kFp8;             // weights are E4M3 codes
     const int K = kMode == 0 ? s.H : s.I;
     const uint64_t w_rows = kMode == 0 ? 2ull * s.I : static_cast<uint64_t>(s.H);
     // weight box rows: Swap-AB gate/up halves (64) or W2 rows (128); normal
@@ -1002,7 +814,7 @@ static cudaError_t run_gemm(const moe_shape_t &s, const GemmArgs &a, cudaStream_
     const uint32_t xbox = kSwap ? 16 : 128;     // Swap-AB loads token rows in 16-row boxes
     CUtensorMap tm_w, tm_x;
     if (!make_map(&tm_w, a.wgt, u8w, Et * w_rows, K, wbox, Cf::kRowBytes) ||
-        !make_map(&tm_x, a.act, u8, a.max_rows, K, xbox, Cf::kRowBytes)) {
+        !make_map(&tm_x, a.act, u8, Cf::kPlanes * a.max_rows, K, xbox, Cf::kRowBytes)) {
         *host_err = MOE_ERR_CUDA;
         return cudaSuccess;
     }
@@ -1020,6 +832,8 @@ static cudaError_t run_gemm(const moe_shape_t &s, const GemmArgs &a, cudaStream_
     p.status = a.status;
     p.counters = a.counters;
     p.partials = a.partials;
+    p.rowscale = a.rowscale;
+    p.lo_rows = static_cast<int>(a.max_rows);
     // decode tiles split cheaply (few token columns); prefill tiles carry
     // 128 KB of fp32 partials, so whole tiles are preferred there
     p.stream_k = kSwap ? 1 : 2;
@@ -1031,8 +845,6 @@ static cudaError_t run_gemm(const moe_shape_t &s, const GemmArgs &a, cudaStream_
     return launch_kernel(kern, dim3(sm_count()), dim3(Cf::kThreads), Cf::kDynSmem, st, a.chained, tm_w, tm_x, p);
 }
 
-int gemm_acc_cols(const GemmPlan &p) { return p.swap ? p.bn : 256; }
-
 cudaError_t launch_grouped_gemm(const moe_shape_t &s, const GemmPlan &p, const GemmArgs &a,
                                 cudaStream_t st, int *launches, int *host_err)
 {
@@ -1041,7 +853,22 @@ cudaError_t launch_grouped_gemm(const moe_shape_t &s, const GemmPlan &p, const G
     const bool w8 = s.wdtype == MOE_E4M3 && s.adtype == MOE_BF16;
     cudaError_t err = cudaSuccess;
     if (w8) {
-#define MOE_W8(MODE, BN) err = run_gemm<MODE, true, false, BN, true>(s, a, st, host_err)
+        // E4M3 weights with bf16 activations: the activation rows are first
+        // split into two E4M3 planes under a per-row power-of-two scale
+        // (v = s * (hi + lo)), then the grouped GEMM runs on the E4M3 tensor
+        // path with both planes stacked in N.
+        if (!a.chained) {
+            err = cudaMemsetAsync(a.counters, 0, 2 * kMaxCtas * sizeof(int32_t), st);
+            if (err != cudaSuccess) return err;
+        }
+        err = launch_split_hilo(s, a.act, a.mode == 0 ? s.H : s.I, a.offsets, a.planes, a.rowscale,
+                                a.max_rows, st, a.chained);
+        if (err != cudaSuccess) return err;
+        *launches += 1;
+        GemmArgs g = a;
+        g.act = a.planes;
+        g.chained = true;          // counters are zero; a dependent launch of the split
+#define MOE_W8(MODE, BN) err = run_gemm<MODE, true, true, BN, true>(s, g, st, host_err)
 #define MOE_W8_BY_BN(MODE)                   \
     switch (p.bn) {                          \
     case 16: MOE_W8(MODE, 16); break;        \

@@ -64,7 +64,8 @@ bool ws_layout(const moe_shape_t &s, WsLayout &L)
     L.max_rows = R + static_cast<int64_t>(s.n_shared) * s.T + static_cast<int64_t>(Et) * (s.pad - 1);
     L.n_chunks = static_cast<int>((R + kAlignChunk - 1) / kAlignChunk);
     const GemmPlan p = plan_gemm(s);
-    L.acc_cols = p.swap ? p.bn : 256;
+    const bool w8 = s.wdtype == MOE_E4M3 && s.adtype == MOE_BF16;
+    L.acc_cols = p.swap ? (w8 ? 2 : 1) * p.bn : 256;
     const size_t ab = s.adtype == MOE_E4M3 ? 1 : 2;
     size_t o = 0;
     L.ctrl = o;        o += up256(sizeof(Ctrl));
@@ -83,6 +84,11 @@ bool ws_layout(const moe_shape_t &s, WsLayout &L)
     L.h = o;           o += up256(L.max_rows * s.I * ab);
     L.y = o;           o += up256(L.max_rows * s.H * 4);
     L.partials = o;    o += up256(static_cast<size_t>(2 * kMaxCtas) * 128 * L.acc_cols * 4);
+    // hi/lo E4M3 planes of GEMM1's then GEMM2's activations (reused: the
+    // split of h runs after GEMM1 has finished reading the planes of xp)
+    const int64_t kmax = s.H > s.I ? s.H : s.I;
+    L.planes = o;      o += w8 ? up256(2 * L.max_rows * kmax) : 0;
+    L.rowscale = o;    o += w8 ? up256(L.max_rows * 4) : 0;
     L.total = o;
     return true;
 }
@@ -210,6 +216,8 @@ static int gemm_common(const moe_shape_t *shape, int mode, const void *act, cons
     a.status = &reinterpret_cast<Ctrl *>(b + L.ctrl)->status;
     a.counters = reinterpret_cast<int32_t *>(b + L.counters);
     a.partials = reinterpret_cast<float *>(b + L.partials);
+    a.planes = b + L.planes;
+    a.rowscale = reinterpret_cast<float *>(b + L.rowscale);
     a.max_rows = L.max_rows;
     int host_err = MOE_OK;
     cudaError_t e = launch_grouped_gemm(*shape, plan_gemm(*shape), a, stream, &g_launches, &host_err);
@@ -298,6 +306,8 @@ int moe_fused_forward(const moe_shape_t *shape, const void *x, const float *logi
     a.status = &ctrl->status;
     a.counters = reinterpret_cast<int32_t *>(b + L.counters);
     a.partials = reinterpret_cast<float *>(b + L.partials);
+    a.planes = b + L.planes;
+    a.rowscale = reinterpret_cast<float *>(b + L.rowscale);
     a.max_rows = L.max_rows;
     a.offsets = offsets;
     int host_err = MOE_OK;

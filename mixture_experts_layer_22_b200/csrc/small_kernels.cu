@@ -7,6 +7,7 @@
 // stresses keeping routing decisions on the GPU, without host-side control
 // flow.  Nothing here reads a routing result on the host.
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_fp8.h>
 
 #include "common.cuh"
@@ -425,6 +426,111 @@ cudaError_t launch_gather(const moe_shape_t &s, const void *x, const int32_t *so
     return launch_kernel(s.adtype == MOE_E4M3 ? gather_kernel<true> : gather_kernel<false>, dim3(blocks),
                          dim3(256), 0, st, chained, static_cast<const uint4 *>(x), sorted_rows, offsets, Et,
                          s.T, s.k, s.H, a1, xp);
+}
+
+// ------------------------------------------------------------------ hi/lo split
+// E4M3 weights with bf16 activations run on the E4M3 tensor path.  Each
+// activation row v (bf16, K values) is written as two E4M3 planes under one
+// power-of-two scale s per row:
+//   hi = e4m3(v / s),  lo = e4m3(v / s - hi),  v = s * (hi + lo).
+// s is the smallest power of two with max|v| <= 448 s, so nothing saturates.
+// A bf16 value has 8 significant bits and hi keeps the top 4 (rounded), so
+// the remainder v/s - hi needs at most 4 bits and is exact in E4M3 whenever
+// it is at least 2^-6 (the smallest normal); smaller remainders round to the
+// 2^-9 subnormal grid.  The split is therefore exact except for elements
+// below about 2^-11 of the row's max magnitude, which are off by at most
+// 2^-10 s (about 4.4e-6 of the row max): far below the bf16 rounding of
+// the GEMM outputs.  Products of E4M3 codes are exact in the fp32
+// accumulator, so the GEMM computes the bf16-activation products.
+__device__ __forceinline__ float e4m3_value(uint32_t code)
+{
+    const __half_raw h = __nv_cvt_fp8_to_halfraw(static_cast<__nv_fp8_storage_t>(code), __NV_E4M3);
+    return __half2float(__half(h));
+}
+
+__device__ __forceinline__ void split8(uint4 d, float inv_s, uint2 &hi, uint2 &lo)
+{
+    const uint32_t wv[4] = {d.x, d.y, d.z, d.w};
+    uint32_t qh[2] = {0, 0}, ql[2] = {0, 0};
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const float v = __uint_as_float(((wv[i >> 1] >> ((i & 1) * 16)) & 0xFFFFu) << 16) * inv_s;
+        const uint32_t ch = __nv_cvt_float_to_fp8(v, __NV_SATFINITE, __NV_E4M3) & 0xFFu;
+        const uint32_t cl = __nv_cvt_float_to_fp8(v - e4m3_value(ch), __NV_SATFINITE, __NV_E4M3) & 0xFFu;
+        qh[i >> 2] |= ch << ((i & 3) * 8);
+        ql[i >> 2] |= cl << ((i & 3) * 8);
+    }
+    hi = make_uint2(qh[0], qh[1]);
+    lo = make_uint2(ql[0], ql[1]);
+}
+
+__device__ __forceinline__ float abs_max8(uint4 d)
+{
+    const uint32_t wv[4] = {d.x, d.y, d.z, d.w};
+    float m = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        m = fmaxf(m, fabsf(__uint_as_float(wv[i] << 16)));
+        m = fmaxf(m, fabsf(__uint_as_float(wv[i] & 0xFFFF0000u)));
+    }
+    return m;
+}
+
+// Exponent e of the row scale s = 2^e: amax = M * 2^E with M in [1, 2);
+// amax <= 448 * 2^e  <=>  e >= E - 8 when M <= 1.75, else e >= E - 7.
+__device__ __forceinline__ int row_scale_exp(float amax)
+{
+    const uint32_t b = __float_as_uint(amax);
+    const int ef = static_cast<int>((b >> 23) & 0xFFu);
+    if (ef == 0) return -126;                         // zero or subnormal max: any scale
+    const int e = (ef - 127) - 8 + ((b & 0x7FFFFFu) > 0x600000u ? 1 : 0);
+    return e < -126 ? -126 : e;
+}
+
+// One block per permuted row (grid-stride over the rows that exist).
+__global__ void __launch_bounds__(256) split_hilo_kernel(const uint4 *__restrict__ src, int K,
+                                                         const int32_t *__restrict__ offsets, int Et,
+                                                         int64_t lo_rows, uint2 *planes, float *scale)
+{
+    grid_dep_wait();
+    grid_dep_launch();
+    __shared__ float s_red[8];
+    const int total = offsets[Et];
+    const int nv = K / 8;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    for (int row = blockIdx.x; row < total; row += gridDim.x) {
+        const uint4 *r = src + static_cast<size_t>(row) * nv;
+        float m = 0.0f;
+        for (int v = threadIdx.x; v < nv; v += blockDim.x) m = fmaxf(m, abs_max8(r[v]));
+        m = warp_max(m);
+        if (lane == 0) s_red[warp] = m;
+        __syncthreads();
+        m = s_red[0];
+#pragma unroll
+        for (int i = 1; i < 8; ++i) m = fmaxf(m, s_red[i]);
+        __syncthreads();                                  // s_red is rewritten by the next row
+        const int e = row_scale_exp(m);
+        const float inv_s = __uint_as_float(static_cast<uint32_t>(127 - e) << 23);   // 2^-e
+        uint2 *ph = planes + static_cast<size_t>(row) * nv;
+        uint2 *pl = planes + static_cast<size_t>(lo_rows + row) * nv;
+        for (int v = threadIdx.x; v < nv; v += blockDim.x) {
+            uint2 hi, lo;
+            split8(r[v], inv_s, hi, lo);
+            ph[v] = hi;
+            pl[v] = lo;
+        }
+        if (threadIdx.x == 0) scale[row] = __uint_as_float(static_cast<uint32_t>(127 + e) << 23);
+    }
+}
+
+cudaError_t launch_split_hilo(const moe_shape_t &s, const void *src, int K, const int32_t *offsets,
+                              void *planes, float *scale, int64_t max_rows, cudaStream_t st, bool chained)
+{
+    int blocks = static_cast<int>(max_rows < 148 * 8 ? max_rows : 148 * 8);
+    if (blocks < 1) blocks = 1;
+    return launch_kernel(split_hilo_kernel, dim3(blocks), dim3(256), 0, st, chained,
+                         static_cast<const uint4 *>(src), K, offsets, s.E + s.n_shared, max_rows,
+                         static_cast<uint2 *>(planes), scale);
 }
 
 // ------------------------------------------------------------------ combine

@@ -366,9 +366,10 @@ def test_fused_fp8_weights_bf16_activations_sigmoid_shared(T):
 @pytest.mark.parametrize("mode", ["swiglu", "down"])
 def test_e4m3_weight_expansion_is_exact(mode):
     """E4M3 weights drawn from every finite code (subnormals included), scale
-    1: the E4M3-weight GEMM must equal the bf16-weight GEMM on the identical
-    bf16 values up to fp32 summation order, which checks that the kernel's
-    E4M3 -> bf16 expansion is exact."""
+    1: the E4M3-weight GEMM (bf16 activations split into hi/lo E4M3 planes)
+    must equal the bf16-weight GEMM on the identical values up to fp32
+    summation order and the split's sub-2^-11 remainders, which checks that
+    every weight code and the activation split are taken exactly."""
     T, H, I, E, k = 32, 512, 256, 4, 2
     rng = np.random.default_rng(12)
     codes = np.array([c for c in range(256) if c not in (0x7F, 0xFF)], dtype=np.uint8)
