@@ -62,10 +62,9 @@ struct GemmParams {
     int stream_k;     // 0: whole tiles only.  Otherwise whole tiles for all but the
                       // last one or two rounds, which are split into equal K-step ranges
                       // (stream-K, each tile shared by at most ~2 CTAs), except that whole
-                      // tiles are used throughout when the last round is full enough:
-                      // 1 (HBM-bound decode): >= 70% of the CTAs busy (an idle SM costs
-                      //   little while the others keep HBM saturated);
-                      // 2 (tensor-bound prefill): rounds >= 90% full on average.
+                      // tiles are used throughout when the rounds are full enough:
+                      // 1 (HBM-bound decode): >= 97% full on average;
+                      // 2 (tensor-bound prefill): >= 90% full on average.
 };
 
 template <int kMode, bool kSwap, bool kFp8, int kBN, bool kHiLo = false>
@@ -84,7 +83,13 @@ struct Cfg {
     static constexpr int kDynBudget = 205 * 1024;
     static constexpr int kStagesRaw = kDynBudget / kStage;
     static constexpr int kStages = kStagesRaw > 12 ? 12 : kStagesRaw;
-    static constexpr int kDynSmem = kStages * kStage + 1024;
+    // Normal order: kStages stages of kStage bytes.  Swap-AB: the stage size
+    // is set per launch from the largest segment (capped at the tile), so a
+    // decode batch whose experts see few rows keeps more stages in flight:
+    // up to kSlots stages in a ring of kRingBytes.
+    static constexpr int kSlots = kSwap ? 12 : kStages;
+    static constexpr int kRingBytes = kSwap ? (kDynBudget / 1024) * 1024 : kStages * kStage;
+    static constexpr int kDynSmem = kRingBytes + 1024;
     // epilogue warps 2 .. 2+kEpiWarps-1; the normal order uses two per
     // tensor-memory lane quarter, each taking half of the tile's columns
     static constexpr int kEpiWarps = kSwap ? 4 : 8;
@@ -99,6 +104,7 @@ struct Cfg {
     // h leaves GEMM1 as E4M3 only on the all-E4M3 path
     static constexpr bool kOutE4M3 = kFp8 && !kHiLo;
     static_assert(kStages >= 2, "smem ring too small");
+    static_assert(!kSwap || kRingBytes >= 2 * kStage, "Swap-AB ring must hold two full-size stages");
     static_assert(!kHiLo || (kSwap && kFp8 && kBN <= 128), "hi/lo planes: Swap-AB on the E4M3 tensor path");
     static_assert(kTmemCols <= 512, "tensor memory");
 };
@@ -243,7 +249,8 @@ __global__ void __launch_bounds__(Cfg<kMode, kSwap, kFp8, kBN, kHiLo>::kThreads,
     extern __shared__ uint8_t dyn_smem[];
     __shared__ int s_off[kMaxExpertsTotal + 1];
     __shared__ int s_prefix[kMaxExpertsTotal + 1];
-    __shared__ __align__(8) uint64_t s_full[C::kStages], s_empty[C::kStages];
+    __shared__ __align__(8) uint64_t s_full[C::kSlots], s_empty[C::kSlots];
+    __shared__ int s_max_seg;
     __shared__ __align__(8) uint64_t s_tfull[2], s_tempty[2], s_drain;
     __shared__ uint32_t s_tmem_base;
     __shared__ volatile int s_abort;
@@ -263,7 +270,7 @@ __global__ void __launch_bounds__(Cfg<kMode, kSwap, kFp8, kBN, kHiLo>::kThreads,
     // ---- set-up: barriers, tensor memory, tile table ----
     if (threadIdx.x == 0) {
         s_abort = 0;
-        for (int i = 0; i < C::kStages; ++i) {
+        for (int i = 0; i < C::kSlots; ++i) {
             mbar_init(smem_u32(&s_full[i]), 1);
             mbar_init(smem_u32(&s_empty[i]), 1);
         }
@@ -288,10 +295,11 @@ __global__ void __launch_bounds__(Cfg<kMode, kSwap, kFp8, kBN, kHiLo>::kThreads,
         __syncwarp();
         const int per = (Et + 31) / 32;
         const int lo = min(Et, lane * per), hi = min(Et, lo + per);
-        int sum = 0;
+        int sum = 0, mx = 0;
         bool bad = false;
         for (int e = lo; e < hi; ++e) {
             const int seg = s_off[e + 1] - s_off[e];
+            mx = max(mx, seg);
             if (seg < 0 || (seg & 15) != 0 || (s_off[e] & 15) != 0) bad = true;
             sum += seg > 0 ? ((seg + C::kRowsTile - 1) / C::kRowsTile) * n_ft : 0;
         }
@@ -308,6 +316,9 @@ __global__ void __launch_bounds__(Cfg<kMode, kSwap, kFp8, kBN, kHiLo>::kThreads,
             run += seg > 0 ? ((seg + C::kRowsTile - 1) / C::kRowsTile) * n_ft : 0;
         }
         if (lane == 31) s_prefix[Et] = inc;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        if (lane == 0) s_max_seg = mx;
         if (__any_sync(0xffffffffu, bad) && lane == 0) {
             set_status(p.status, MOE_ERR_DEVICE_CHECK);
             s_prefix[Et] = 0;   // no work: refuse mis-aligned segments
@@ -318,16 +329,27 @@ __global__ void __launch_bounds__(Cfg<kMode, kSwap, kFp8, kBN, kHiLo>::kThreads,
     tc_fence_after();
     const uint32_t tmem_base = s_tmem_base;
 
+    // ring geometry of this launch (Swap-AB: room for the largest tile's rows)
+    const int tile_rows_max = max(16, min(C::kRowsTile, s_max_seg));
+    const int stage_bytes = kSwap ? C::kStageA + C::kPlanes * tile_rows_max * C::kRowBytes : C::kStage;
+    const int n_stages = kSwap ? min(C::kSlots, C::kRingBytes / stage_bytes) : C::kStages;
+
     Sched S;
     S.n_tiles = s_prefix[Et];
     S.KT = p.K / C::kKStage;
     S.G = gridDim.x;
     const int rem = S.n_tiles % S.G;
+    // whole tiles throughout when the idle share of the last round, over
+    // all rounds, is small: 3% for decode (each SM streams at a bounded
+    // rate, so idle SMs cost time) and 10% for prefill (split tiles carry
+    // 128 KB partials)
+    const int rounds = (S.n_tiles + S.G - 1) / S.G;
+    const long long idle = static_cast<long long>(S.G) * rounds - S.n_tiles;
     const bool full_enough = S.n_tiles >= S.G &&
-                             10 * S.n_tiles >= 9 * S.G * ((S.n_tiles + S.G - 1) / S.G);
+                             100 * idle <= (p.stream_k == 1 ? 3LL : 10LL) * S.G * rounds;
     if (!p.stream_k || rem == 0) S.dp_tiles = S.n_tiles;
     else if (S.n_tiles < S.G) S.dp_tiles = 0;
-    else if ((p.stream_k == 1 && 10 * rem >= 7 * S.G) || (p.stream_k == 2 && full_enough)) S.dp_tiles = S.n_tiles;
+    else if (full_enough) S.dp_tiles = S.n_tiles;
     else S.dp_tiles = (S.n_tiles / S.G - 1) * S.G;
     S.sk_tiles = S.n_tiles - S.dp_tiles;
     S.sk_total = static_cast<long long>(S.sk_tiles) * S.KT;
@@ -345,9 +367,9 @@ __global__ void __launch_bounds__(Cfg<kMode, kSwap, kFp8, kBN, kHiLo>::kThreads,
         iter_init(I, S, blockIdx.x);
         Item it;
         int n = 0;
-        while (n < C::kStages && iter_next<C::kRowsTile>(I, S, s_prefix, s_off, Et, n_ft, it)) {
+        while (n < n_stages && iter_next<C::kRowsTile>(I, S, s_prefix, s_off, Et, n_ft, it)) {
             const int wbase = it.e * p.w_rows;
-            for (int kk = it.kb; kk < it.ke && n < C::kStages; ++kk, ++n) {
+            for (int kk = it.kb; kk < it.ke && n < n_stages; ++kk, ++n) {
                 const int kx = kk * C::kKStage;
                 if (kMode == 0) {
                     tma_prefetch_l2_2d(&tm_w, kx, wbase + it.ft * kHalf);
@@ -391,7 +413,7 @@ __global__ void __launch_bounds__(Cfg<kMode, kSwap, kFp8, kBN, kHiLo>::kThreads,
                     // Swap-AB: only the tile's own token rows (16-row boxes), of
                     // both planes for kHiLo
                     mbar_arrive_expect_tx(fb, kSwap ? C::kStageA + C::kPlanes * rows * C::kRowBytes : C::kStage);
-                    const uint32_t sa = smem_u32(tiles + stage * C::kStage);
+                    const uint32_t sa = smem_u32(tiles + stage * stage_bytes);
                     const uint32_t sb = sa + C::kStageA;
                     const int kx = kk * C::kKStage;
                     if (kSwap) {
@@ -416,13 +438,13 @@ __global__ void __launch_bounds__(Cfg<kMode, kSwap, kFp8, kBN, kHiLo>::kThreads,
                         }
                     }
                     ++in_flight;
-                    if (++stage == C::kStages) {
+                    if (++stage == n_stages) {
                         stage = 0;
                         phase ^= 1u;
                     }
                 }
             }
-            if (!ok) drain_ring(s_full, C::kStages, stage, phase, in_flight);   // let issued copies land
+            if (!ok) drain_ring(s_full, n_stages, stage, phase, in_flight);   // let issued copies land
         }
     } else if (warp == 1) {
         // ================= MMA issuer =================
@@ -451,7 +473,7 @@ __global__ void __launch_bounds__(Cfg<kMode, kSwap, kFp8, kBN, kHiLo>::kThreads,
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t sa = smem_u32(tiles + stage * C::kStage);
+                    const uint32_t sa = smem_u32(tiles + stage * stage_bytes);
                     const uint32_t sb = sa + C::kStageA;
 #pragma unroll
                     for (int s = 0; s < C::kMmaPerStage; ++s) {
@@ -462,7 +484,7 @@ __global__ void __launch_bounds__(Cfg<kMode, kSwap, kFp8, kBN, kHiLo>::kThreads,
                         else mma_bf16(d, ad, bd, idesc, accum);
                     }
                     mma_commit(smem_u32(&s_empty[stage]));
-                    if (++stage == C::kStages) {
+                    if (++stage == n_stages) {
                         stage = 0;
                         phase ^= 1u;
                     }
