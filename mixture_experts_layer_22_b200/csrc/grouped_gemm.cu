@@ -67,7 +67,7 @@ struct GemmParams {
                       // 2 (tensor-bound prefill): >= 90% full on average.
 };
 
-template <int kMode, bool kSwap, bool kFp8, int kBN, bool kHiLo = false>
+template <int kMode, bool kSwap, bool kFp8, int kBN, bool kHiLo = false, bool kPair = false>
 struct Cfg {
     // K bytes per operand row and stage (128: the 128-byte swizzle; 64-byte
     // rows with the 64-byte swizzle are supported by the loads and
@@ -97,7 +97,8 @@ struct Cfg {
     static constexpr int kThreads = 64 + kEpiThreads;
     static constexpr int kAccCols = kSwap ? kPlanes * kBN : 256;   // fp32 columns per accumulator
     static constexpr int kTmemCols = (2 * kAccCols) <= 32 ? 32 : 2 * kAccCols;
-    static constexpr int kRowsTile = kSwap ? kBN : 128;     // token rows per tile
+    // token rows per tile (kPair: a CTA pair's tile, 128 rows in each CTA)
+    static constexpr int kRowsTile = kSwap ? kBN : (kPair ? 256 : 128);
     static constexpr int kFeatTile = kMode == 0 ? (kSwap ? 64 : 128) : (kSwap ? 128 : 256);
     static constexpr int kKStage = kFp8 ? kRowBytes : kRowBytes / 2;   // K elements per work step
     static constexpr uint32_t kFmt = kFp8 ? 0u : 1u;
@@ -106,6 +107,10 @@ struct Cfg {
     static_assert(kStages >= 2, "smem ring too small");
     static_assert(!kSwap || kRingBytes >= 2 * kStage, "Swap-AB ring must hold two full-size stages");
     static_assert(!kHiLo || (kSwap && kFp8 && kBN <= 128), "hi/lo planes: Swap-AB on the E4M3 tensor path");
+    // kPair: normal order on a CTA pair (tcgen05 .cta_group::2): M = 256 token
+    // rows (128 per CTA), N = 256 weight rows (each CTA stages its 128), each
+    // CTA's tensor memory holds its 128 rows x 256 columns
+    static_assert(!kPair || (!kSwap && !kHiLo && kBN == 128), "CTA pairs: normal order, 128-row B halves");
     static_assert(kTmemCols <= 512, "tensor memory");
 };
 
@@ -240,12 +245,12 @@ __device__ __forceinline__ void drain_ring(uint64_t *full, int nstages, int stag
     }
 }
 
-template <int kMode, bool kSwap, bool kFp8, int kBN, bool kHiLo = false>
-__global__ void __launch_bounds__(Cfg<kMode, kSwap, kFp8, kBN, kHiLo>::kThreads, 1)
+template <int kMode, bool kSwap, bool kFp8, int kBN, bool kHiLo = false, bool kPair = false>
+__global__ void __launch_bounds__(Cfg<kMode, kSwap, kFp8, kBN, kHiLo, kPair>::kThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tm_w,
                         const __grid_constant__ CUtensorMap tm_x, GemmParams p)
 {
-    using C = Cfg<kMode, kSwap, kFp8, kBN, kHiLo>;
+    using C = Cfg<kMode, kSwap, kFp8, kBN, kHiLo, kPair>;
     extern __shared__ uint8_t dyn_smem[];
     __shared__ int s_off[kMaxExpertsTotal + 1];
     __shared__ int s_prefix[kMaxExpertsTotal + 1];
@@ -264,6 +269,9 @@ __global__ void __launch_bounds__(Cfg<kMode, kSwap, kFp8, kBN, kHiLo>::kThreads,
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int Et = p.E_tot;
+    // kPair: CTA `rank` of the pair; the pair is one unit of the tile schedule
+    const uint32_t rank = kPair ? cluster_ctarank() : 0u;
+    const int unit = kPair ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
     uint8_t *tiles = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(dyn_smem) + 1023) &
                                                  ~static_cast<uintptr_t>(1023));
 
@@ -276,7 +284,8 @@ __global__ void __launch_bounds__(Cfg<kMode, kSwap, kFp8, kBN, kHiLo>::kThreads,
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(smem_u32(&s_tfull[i]), 1);
-            mbar_init(smem_u32(&s_tempty[i]), C::kEpiWarps);
+            // kPair: rank 0's accumulator barrier also counts the peer's epilogue warps
+            mbar_init(smem_u32(&s_tempty[i]), (kPair ? 2 : 1) * C::kEpiWarps);
         }
         mbar_init(smem_u32(&s_drain), 1);
         fence_mbar_init();
@@ -284,8 +293,13 @@ __global__ void __launch_bounds__(Cfg<kMode, kSwap, kFp8, kBN, kHiLo>::kThreads,
         prefetch_tmap(&tm_x);
     }
     if (warp == 1) {
-        tmem_alloc(smem_u32(&s_tmem_base), C::kTmemCols);
-        tmem_relinquish();
+        if constexpr (kPair) {
+            tmem_alloc_pair(smem_u32(&s_tmem_base), C::kTmemCols);
+            tmem_relinquish_pair();
+        } else {
+            tmem_alloc(smem_u32(&s_tmem_base), C::kTmemCols);
+            tmem_relinquish();
+        }
     }
     const int n_ft = (p.n_feat + C::kFeatTile - 1) / C::kFeatTile;
     if (warp == 2) {
@@ -326,6 +340,7 @@ __global__ void __launch_bounds__(Cfg<kMode, kSwap, kFp8, kBN, kHiLo>::kThreads,
     }
     tc_fence_before();
     __syncthreads();
+    if constexpr (kPair) cluster_sync();   // the peer's barriers exist before any signal crosses
     tc_fence_after();
     const uint32_t tmem_base = s_tmem_base;
 
@@ -337,7 +352,7 @@ __global__ void __launch_bounds__(Cfg<kMode, kSwap, kFp8, kBN, kHiLo>::kThreads,
     Sched S;
     S.n_tiles = s_prefix[Et];
     S.KT = p.K / C::kKStage;
-    S.G = gridDim.x;
+    S.G = kPair ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
     const int rem = S.n_tiles % S.G;
     // whole tiles throughout when the idle share of the last round, over
     // all rounds, is small: 3% for decode (each SM streams at a bounded
@@ -364,14 +379,18 @@ __global__ void __launch_bounds__(Cfg<kMode, kSwap, kFp8, kBN, kHiLo>::kThreads,
     if (warp == 0 && lane == 0 && p.pdl) {
         constexpr int kHalf = kSwap ? 64 : 128;   // weight rows per gate/up half-tile
         ItemIter I;
-        iter_init(I, S, blockIdx.x);
+        iter_init(I, S, unit);
         Item it;
         int n = 0;
         while (n < n_stages && iter_next<C::kRowsTile>(I, S, s_prefix, s_off, Et, n_ft, it)) {
             const int wbase = it.e * p.w_rows;
             for (int kk = it.kb; kk < it.ke && n < n_stages; ++kk, ++n) {
                 const int kx = kk * C::kKStage;
-                if (kMode == 0) {
+                if (kPair) {
+                    // this CTA's half: gate (rank 0) or up (rank 1) rows; W2 rows [128 rank, +128)
+                    tma_prefetch_l2_2d(&tm_w, kx, kMode == 0 ? wbase + (rank ? p.n_feat : 0) + it.ft * 128
+                                                             : wbase + it.ft * 256 + 128 * static_cast<int>(rank));
+                } else if (kMode == 0) {
                     tma_prefetch_l2_2d(&tm_w, kx, wbase + it.ft * kHalf);
                     tma_prefetch_l2_2d(&tm_w, kx, wbase + p.n_feat + it.ft * kHalf);
                 } else {
@@ -397,7 +416,7 @@ __global__ void __launch_bounds__(Cfg<kMode, kSwap, kFp8, kBN, kHiLo>::kThreads,
             uint32_t phase = 0;
             int in_flight = 0;
             ItemIter I;
-            iter_init(I, S, blockIdx.x);
+            iter_init(I, S, unit);
             Item it;
             bool ok = true;
             while (ok && iter_next<C::kRowsTile>(I, S, s_prefix, s_off, Et, n_ft, it)) {
@@ -411,8 +430,11 @@ __global__ void __launch_bounds__(Cfg<kMode, kSwap, kFp8, kBN, kHiLo>::kThreads,
                     }
                     const uint32_t fb = smem_u32(&s_full[stage]);
                     // Swap-AB: only the tile's own token rows (16-row boxes), of
-                    // both planes for kHiLo
-                    mbar_arrive_expect_tx(fb, kSwap ? C::kStageA + C::kPlanes * rows * C::kRowBytes : C::kStage);
+                    // both planes for kHiLo.  kPair: rank 0's barrier counts the
+                    // bytes of both CTAs.
+                    if (!kPair || rank == 0)
+                        mbar_arrive_expect_tx(fb, kSwap ? C::kStageA + C::kPlanes * rows * C::kRowBytes
+                                                        : (kPair ? 2 : 1) * C::kStage);
                     const uint32_t sa = smem_u32(tiles + stage * stage_bytes);
                     const uint32_t sb = sa + C::kStageA;
                     const int kx = kk * C::kKStage;
@@ -428,6 +450,15 @@ __global__ void __launch_bounds__(Cfg<kMode, kSwap, kFp8, kBN, kHiLo>::kThreads,
                         if (kHiLo)
                             for (int rr = 0; rr < rows; rr += 16)
                                 tma_load_2d(sb + (rows + rr) * C::kRowBytes, &tm_x, fb, kx, p.lo_rows + row0 + rr, pol_x);
+                    } else if (kPair) {
+                        // this CTA's 128 token rows and its half of the 256 weight
+                        // rows (gate or up rows of 128 features; W2 rows [128 rank, +128))
+                        const uint32_t fb0 = mapa_shared(fb, 0);
+                        tma_load_2d_pair(sa, &tm_x, fb0, kx, row0 + 128 * static_cast<int>(rank), pol_x);
+                        tma_load_2d_pair(sb, &tm_w, fb0, kx,
+                                         kMode == 0 ? wbase + (rank ? p.n_feat : 0) + it.ft * 128
+                                                    : wbase + it.ft * 256 + 128 * static_cast<int>(rank),
+                                         pol_w);
                     } else {
                         tma_load_2d(sa, &tm_x, fb, kx, row0, pol_x);
                         if (kMode == 0) {
@@ -444,21 +475,33 @@ __global__ void __launch_bounds__(Cfg<kMode, kSwap, kFp8, kBN, kHiLo>::kThreads,
                     }
                 }
             }
-            if (!ok) drain_ring(s_full, n_stages, stage, phase, in_flight);   // let issued copies land
+            if (!ok) {
+                // let issued copies land (kPair: rank 1's copies complete on rank
+                // 0's barriers; the pair waits out its copies at tear-down)
+                if (!kPair || rank == 0) drain_ring(s_full, n_stages, stage, phase, in_flight);
+            } else if (kPair) {
+                // every stage this CTA filled has been consumed, so no commit of
+                // rank 0's MMAs is still on its way to this CTA's barriers
+                drain_ring(s_empty, n_stages, stage, phase, in_flight);
+            }
         }
     } else if (warp == 1) {
-        // ================= MMA issuer =================
-        if (lane == 0) {
+        // ================= MMA issuer (kPair: rank 0 only) =================
+        if (lane == 0 && (!kPair || rank == 0)) {
             int stage = 0;
             uint32_t phase = 0;
             int acc = 0;
             uint32_t acc_phase = 0;
             ItemIter I;
-            iter_init(I, S, blockIdx.x);
+            iter_init(I, S, unit);
             Item it;
             bool ok = true;
+            // kPair: both barriers below also receive the peer CTA's arrivals
+            auto wait_bar = [&](uint32_t bar, uint32_t parity) -> bool {
+                return kPair ? mbar_wait_cluster(bar, parity, &s_abort) : mbar_wait(bar, parity, &s_abort);
+            };
             while (ok && iter_next<C::kRowsTile>(I, S, s_prefix, s_off, Et, n_ft, it)) {
-                if (!mbar_wait(smem_u32(&s_tempty[acc]), acc_phase ^ 1u, &s_abort)) break;
+                if (!wait_bar(smem_u32(&s_tempty[acc]), acc_phase ^ 1u)) break;
                 tc_fence_after();
                 const uint32_t d = tmem_base + acc * C::kAccCols;
                 int n = 256;
@@ -466,9 +509,9 @@ __global__ void __launch_bounds__(Cfg<kMode, kSwap, kFp8, kBN, kHiLo>::kThreads,
                     const int seg = s_off[it.e + 1] - s_off[it.e];
                     n = C::kPlanes * min(C::kRowsTile, seg - it.rt * C::kRowsTile);
                 }
-                const uint32_t idesc = idesc_make(C::kFmt, 128, n);
+                const uint32_t idesc = idesc_make(C::kFmt, kPair ? 256 : 128, n);
                 for (int kk = it.kb; kk < it.ke; ++kk) {
-                    if (!mbar_wait(smem_u32(&s_full[stage]), phase, &s_abort)) {
+                    if (!wait_bar(smem_u32(&s_full[stage]), phase)) {
                         ok = false;
                         break;
                     }
@@ -480,24 +523,33 @@ __global__ void __launch_bounds__(Cfg<kMode, kSwap, kFp8, kBN, kHiLo>::kThreads,
                         const uint64_t ad = C::kRowBytes == 128 ? sdesc_k_sw128(sa + s * 32) : sdesc_k_sw64(sa + s * 32);
                         const uint64_t bd = C::kRowBytes == 128 ? sdesc_k_sw128(sb + s * 32) : sdesc_k_sw64(sb + s * 32);
                         const uint32_t accum = (kk > it.kb || s > 0) ? 1u : 0u;
-                        if (kFp8) mma_e4m3(d, ad, bd, idesc, accum);
-                        else mma_bf16(d, ad, bd, idesc, accum);
+                        if constexpr (kPair) {
+                            if (kFp8) mma_e4m3_pair(d, ad, bd, idesc, accum);
+                            else mma_bf16_pair(d, ad, bd, idesc, accum);
+                        } else {
+                            if (kFp8) mma_e4m3(d, ad, bd, idesc, accum);
+                            else mma_bf16(d, ad, bd, idesc, accum);
+                        }
                     }
-                    mma_commit(smem_u32(&s_empty[stage]));
+                    // kPair: the stage is free in both CTAs
+                    if constexpr (kPair) mma_commit_pair(smem_u32(&s_empty[stage]), 3);
+                    else mma_commit(smem_u32(&s_empty[stage]));
                     if (++stage == n_stages) {
                         stage = 0;
                         phase ^= 1u;
                     }
                 }
                 if (!ok) break;
-                mma_commit(smem_u32(&s_tfull[acc]));
+                if constexpr (kPair) mma_commit_pair(smem_u32(&s_tfull[acc]), 3);   // both epilogues
+                else mma_commit(smem_u32(&s_tfull[acc]));
                 if (++acc == 2) {
                     acc = 0;
                     acc_phase ^= 1u;
                 }
             }
             // every MMA issued above has completed once this barrier fires
-            mma_commit(smem_u32(&s_drain));
+            if constexpr (kPair) mma_commit_pair(smem_u32(&s_drain), 1);
+            else mma_commit(smem_u32(&s_drain));
             volatile int no_abort = 0;
             mbar_wait(smem_u32(&s_drain), 0, &no_abort);
         }
@@ -511,15 +563,18 @@ __global__ void __launch_bounds__(Cfg<kMode, kSwap, kFp8, kBN, kHiLo>::kThreads,
         int acc = 0;
         uint32_t acc_phase = 0;
         ItemIter I;
-        iter_init(I, S, blockIdx.x);
+        iter_init(I, S, unit);
         Item it;
         while (iter_next<C::kRowsTile>(I, S, s_prefix, s_off, Et, n_ft, it)) {
-            const bool got = mbar_wait(smem_u32(&s_tfull[acc]), acc_phase, &s_abort);
+            const bool got = kPair ? mbar_wait_cluster(smem_u32(&s_tfull[acc]), acc_phase, &s_abort)
+                                   : mbar_wait(smem_u32(&s_tfull[acc]), acc_phase, &s_abort);
             if (!named_bar_and(1, C::kEpiThreads, got)) break;   // all epilogue warps agree
             tc_fence_after();
             const int seg = s_off[it.e + 1] - s_off[it.e];
-            const int row0 = s_off[it.e] + it.rt * C::kRowsTile;
-            const int rows = min(C::kRowsTile, seg - it.rt * C::kRowsTile);
+            // kPair: this CTA holds rows [128 rank, 128 rank + 128) of the pair's tile
+            const int row0 = s_off[it.e] + it.rt * C::kRowsTile + (kPair ? 128 * static_cast<int>(rank) : 0);
+            const int rows = kPair ? max(0, min(128, seg - it.rt * C::kRowsTile - 128 * static_cast<int>(rank)))
+                                   : min(C::kRowsTile, seg - it.rt * C::kRowsTile);
             // output scale of the tile; kHiLo: times the activation row's own
             // scale (column j of a Swap-AB tile is permuted row row0 + j)
             const float sc = (kHiLo ? 1.0f : p.ascale) * (p.wscale ? __ldg(&p.wscale[it.e]) : 1.0f);
@@ -658,7 +713,11 @@ __global__ void __launch_bounds__(Cfg<kMode, kSwap, kFp8, kBN, kHiLo>::kThreads,
                 }
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(smem_u32(&s_tempty[acc]));
+                if (lane == 0) {
+                    // kPair: the accumulator is free once both CTAs' epilogues are done
+                    if constexpr (kPair) mbar_arrive_cluster(mapa_shared(smem_u32(&s_tempty[acc]), 0));
+                    else mbar_arrive(smem_u32(&s_tempty[acc]));
+                }
             } else {
                 // ---- one share of a split tile: store the raw partial ----
                 float *slot = p.partials + static_cast<size_t>(it.slot) * 128 * C::kAccCols;
@@ -756,10 +815,21 @@ __global__ void __launch_bounds__(Cfg<kMode, kSwap, kFp8, kBN, kHiLo>::kThreads,
     // ---- tear-down ----
     tc_fence_before();
     __syncthreads();
+    if constexpr (kPair) {
+        // After an abort, copies issued by this CTA may still be landing in its
+        // shared memory (their completion was signalled to rank 0): give them
+        // time.  Then neither CTA leaves while the other may still signal it.
+        if (s_abort) {
+            const uint64_t t0 = globaltimer();
+            while (globaltimer() - t0 < 200000ull) {}
+        }
+        cluster_sync();
+    }
     if (threadIdx.x == 0 && s_abort) set_status(p.status, MOE_ERR_TIMEOUT);
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem_base, C::kTmemCols);
+        if constexpr (kPair) tmem_dealloc_pair(tmem_base, C::kTmemCols);
+        else tmem_dealloc(tmem_base, C::kTmemCols);
     }
 }
 
@@ -816,11 +886,39 @@ static int sm_count()
     return n;
 }
 
-template <int kMode, bool kSwap, bool kFp8, int kBN, bool kHiLo = false>
+// Persistent grid of CTA pairs for the kPair kernel: as many pairs as can be
+// resident at once (two SMs of one GPC each), at most half the SM count.
+template <typename Kern>
+static int pair_grid(Kern kern, int threads, int smem)
+{
+    static int grid = 0;
+    if (grid == 0) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(2 * (sm_count() / 2));
+        cfg.blockDim = dim3(threads);
+        cfg.dynamicSmemBytes = smem;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 2;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        int clusters = 0;
+        if (cudaOccupancyMaxActiveClusters(&clusters, kern, &cfg) != cudaSuccess || clusters <= 0) {
+            cudaGetLastError();
+            clusters = 1;
+        }
+        grid = 2 * (clusters < sm_count() / 2 ? clusters : sm_count() / 2);
+    }
+    return grid;
+}
+
+template <int kMode, bool kSwap, bool kFp8, int kBN, bool kHiLo = false, bool kPair = false>
 static cudaError_t run_gemm(const moe_shape_t &s, const GemmArgs &a, cudaStream_t st, int *host_err)
 {
-    using Cf = Cfg<kMode, kSwap, kFp8, kBN, kHiLo>;
-    auto kern = grouped_gemm_kernel<kMode, kSwap, kFp8, kBN, kHiLo>;
+    using Cf = Cfg<kMode, kSwap, kFp8, kBN, kHiLo, kPair>;
+    auto kern = grouped_gemm_kernel<kMode, kSwap, kFp8, kBN, kHiLo, kPair>;
     static std::once_flag once;
     std::call_once(once, [&] {
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cf::kDynSmem);
@@ -831,8 +929,8 @@ static cudaError_t run_gemm(const moe_shape_t &s, const GemmArgs &a, cudaStream_
     const int K = kMode == 0 ? s.H : s.I;
     const uint64_t w_rows = kMode == 0 ? 2ull * s.I : static_cast<uint64_t>(s.H);
     // weight box rows: Swap-AB gate/up halves (64) or W2 rows (128); normal
-    // gate/up halves (128) or W2 rows (256)
-    const uint32_t wbox = kSwap ? (kMode == 0 ? 64 : 128) : (kMode == 0 ? 128 : 256);
+    // gate/up halves (128) or W2 rows (256); a CTA of a pair: 128
+    const uint32_t wbox = kSwap ? (kMode == 0 ? 64 : 128) : (kMode == 0 || kPair ? 128 : 256);
     const uint32_t xbox = kSwap ? 16 : 128;     // Swap-AB loads token rows in 16-row boxes
     CUtensorMap tm_w, tm_x;
     if (!make_map(&tm_w, a.wgt, u8w, Et * w_rows, K, wbox, Cf::kRowBytes) ||
@@ -857,14 +955,33 @@ static cudaError_t run_gemm(const moe_shape_t &s, const GemmArgs &a, cudaStream_
     p.rowscale = a.rowscale;
     p.lo_rows = static_cast<int>(a.max_rows);
     // decode tiles split cheaply (few token columns); prefill tiles carry
-    // 128 KB of fp32 partials, so whole tiles are preferred there
-    p.stream_k = kSwap ? 1 : 2;
+    // 128 KB of fp32 partials, so whole tiles are preferred there; CTA pairs
+    // take whole tiles only
+    p.stream_k = kSwap ? 1 : (kPair ? 0 : 2);
     p.pdl = a.chained ? 1 : 0;
     if (!a.chained) {
         cudaError_t err = cudaMemsetAsync(a.counters, 0, 2 * kMaxCtas * sizeof(int32_t), st);
         if (err != cudaSuccess) return err;
     }
-    return launch_kernel(kern, dim3(sm_count()), dim3(Cf::kThreads), Cf::kDynSmem, st, a.chained, tm_w, tm_x, p);
+    if constexpr (kPair) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(pair_grid(kern, Cf::kThreads, Cf::kDynSmem));
+        cfg.blockDim = dim3(Cf::kThreads);
+        cfg.dynamicSmemBytes = Cf::kDynSmem;
+        cfg.stream = st;
+        cudaLaunchAttribute attr[2];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 2;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[1].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = a.chained ? 2 : 1;
+        return cudaLaunchKernelEx(&cfg, kern, tm_w, tm_x, p);
+    } else {
+        return launch_kernel(kern, dim3(sm_count()), dim3(Cf::kThreads), Cf::kDynSmem, st, a.chained, tm_w, tm_x, p);
+    }
 }
 
 cudaError_t launch_grouped_gemm(const moe_shape_t &s, const GemmPlan &p, const GemmArgs &a,
@@ -919,12 +1036,16 @@ cudaError_t launch_grouped_gemm(const moe_shape_t &s, const GemmPlan &p, const G
             if (fp8) { MOE_BY_BN(1, true) } else { MOE_BY_BN(1, false) }
         }
     } else {
+        // Normal order.  The down projection runs on CTA pairs (256 x 256
+        // tiles, half the weight bytes staged per SM); the gate/up GEMM keeps
+        // one-CTA 128-row tiles: with many small experts the pairs' 256-row
+        // tiles pad more rows than their operand savings gain back (measured).
         if (a.mode == 0) {
             if (fp8) MOE_G(0, false, true, 256);
             else MOE_G(0, false, false, 256);
         } else {
-            if (fp8) MOE_G(1, false, true, 256);
-            else MOE_G(1, false, false, 256);
+            if (fp8) err = run_gemm<1, false, true, 128, false, true>(s, a, st, host_err);
+            else err = run_gemm<1, false, false, 128, false, true>(s, a, st, host_err);
         }
     }
 #undef MOE_BY_BN
