@@ -142,14 +142,20 @@ def tokens(wl: Workload) -> np.ndarray:
     return to_bf16_bits(_normal(wl.seed, "x", 0, (wl.T, wl.H), 1.0))
 
 
+def router_weight(wl: Workload) -> np.ndarray:
+    """Router (gate) weight W_g [E, H], bf16 bits, std 0.02."""
+    return to_bf16_bits(_normal(wl.seed, "w_gate", 0, (wl.E, wl.H), 0.02))
+
+
 def router_logits(wl: Workload, x_bits: np.ndarray) -> np.ndarray:
-    """Router logits [T, E] fp32 (an input of the layer)."""
+    """Router logits [T, E] fp32 (an input of the layer): x . W_g^T summed in
+    double by numpy, or for the Zipf workload N(0,1) noise plus a Zipf bias."""
     if wl.logits == "zipf":
         n = _normal(wl.seed, "logit_noise", 0, (wl.T, wl.E), 1.0).astype(np.float64)
         r = np.arange(1, wl.E + 1, dtype=np.float64) ** (-wl.zipf_s)
         bias = np.log(r / r.sum())
         return (n + bias[None, :]).astype(np.float32)
-    wg = to_bf16_bits(_normal(wl.seed, "w_gate", 0, (wl.E, wl.H), 0.02))
+    wg = router_weight(wl)
     xd = bf16_bits_to_f32(x_bits).astype(np.float64)
     wd = bf16_bits_to_f32(wg).astype(np.float64)
     return (xd @ wd.T).astype(np.float32)

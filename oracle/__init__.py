@@ -56,6 +56,8 @@ def _load():
             lib.orc_bf16_encode.argtypes = [d]
             lib.orc_quant_e4m3_f32.restype = None
             lib.orc_quant_e4m3_f32.argtypes = [P, f, P, l]
+            lib.orc_router_logits.restype = None
+            lib.orc_router_logits.argtypes = [i, i, i, P, P, P]
             lib.orc_route.restype = None
             lib.orc_route.argtypes = [i, i, i, i, i, d, P, P, P]
             lib.orc_align.restype = l
@@ -125,6 +127,20 @@ def quant_e4m3_f32(values, scale: float) -> np.ndarray:
 
 
 # ---------------------------------------------------------------- routing
+def router_logits(x_bits, wg_bits) -> np.ndarray:
+    """Router logits [T, E] fp32 from x [T, H] and Wg [E, H] (bf16 bits), in
+    the fixed summation order the C function documents."""
+    xb = _c(x_bits, np.uint16)
+    wb = _c(wg_bits, np.uint16)
+    T, H = xb.shape
+    E = wb.shape[0]
+    if wb.shape[1] != H or H % 8:
+        raise ValueError("x [T,H] and Wg [E,H] with H a multiple of 8 expected")
+    out = np.empty((T, E), dtype=np.float32)
+    _load().orc_router_logits(T, E, H, _p(xb), _p(wb), _p(out))
+    return out
+
+
 def route(logits, k: int, gate: int = SOFTMAX, renorm: bool = True, routed_scale: float = 1.0):
     lg = _c(logits, np.float32)
     T, E = lg.shape

@@ -149,6 +149,38 @@ static double decode_w(const void *base, int dtype, long idx)
 /* routing: top-k gating over router logits                                  */
 /* ------------------------------------------------------------------------ */
 
+/* Router logits, the step before top-k gating: l[t,e] = sum_h x[t,h] * Wg[e,h]
+ * with x [T,H] and Wg [E,H] bf16.  The Chinese retelling (section
+ * "2. 用于FP8量化的Triton后端路由") has the routing decided inside the fused
+ * kernel, without host control flow; the pages give no summation order.  So
+ * that routing is bit-exact between implementations, the order is fixed as
+ * part of the definition:
+ *   - in double precision (a product of two bf16 values is exact in double);
+ *   - 32 partial sums s_l, l = 0..31: s_l sums, in ascending h, the products
+ *     whose 8-element chunk index h / 8 is congruent to l mod 32;
+ *   - then s_l <- s_l + s_(l xor o) for o = 16, 8, 4, 2, 1 (every s_l ends
+ *     equal);
+ *   - the result rounded once to fp32, to nearest even.
+ * Requires H to be a multiple of 8. */
+void orc_router_logits(int T, int E, int H, const uint16_t *x, const uint16_t *wg, float *logits)
+{
+    for (int t = 0; t < T; ++t)
+        for (int e = 0; e < E; ++e) {
+            double s[32], n[32];
+            for (int l = 0; l < 32; ++l) s[l] = 0.0;
+            for (int c = 0; c < H / 8; ++c)
+                for (int i = 0; i < 8; ++i) {
+                    const long h = 8L * c + i;
+                    s[c % 32] += orc_bf16_decode(x[(long)t * H + h]) * orc_bf16_decode(wg[(long)e * H + h]);
+                }
+            for (int o = 16; o >= 1; o >>= 1) {
+                for (int l = 0; l < 32; ++l) n[l] = s[l] + s[l ^ o];
+                for (int l = 0; l < 32; ++l) s[l] = n[l];
+            }
+            logits[(long)t * E + e] = (float)s[0];
+        }
+}
+
 /* Expert a ranks above expert b: larger logit, equal logits -> lower id.
  * NaN ranks below every number (and among NaNs the lower id first). */
 static int ranks_above(const float *l, int a, int b)

@@ -305,3 +305,69 @@ def test_fp8_activation_quantisation_path():
     out_q = orc.forward(d["x"], d["logits"], d["w13"], d["w2"], E=4, k=2, adtype=orc.E4M3, a1=a1, a2=a2)
     err = np.abs(out_q - out_ref).max() / np.sqrt(np.mean(out_ref ** 2))
     assert 0 < err < 0.2
+
+
+# ------------------------------------------------------------------ router logits
+def _bf16(values) -> np.ndarray:
+    return syn.to_bf16_bits(np.asarray(values, dtype=np.float32))
+
+
+def test_router_logits_one_hot_picks_the_gate_column():
+    """x_t = unit vector at h_t: l[t,e] = Wg[e, h_t] exactly, for positions in
+    every lane and chunk of the fixed order (catches a dropped term, a wrong
+    index or a transposed operand)."""
+    T, E, H = 40, 5, 512
+    rng = np.random.default_rng(21)
+    wg = _bf16(rng.standard_normal((E, H)) * 0.02)
+    hs = rng.choice(H, size=T, replace=False)
+    x = np.zeros((T, H), dtype=np.float32)
+    x[np.arange(T), hs] = 1.0
+    lg = orc.router_logits(_bf16(x), wg)
+    assert np.array_equal(lg, syn.bf16_bits_to_f32(wg)[:, hs].T)
+
+
+def test_router_logits_within_rounding_of_the_exact_sum():
+    """Against the exact rational sum: off by at most the double summation
+    error plus half an fp32 ulp."""
+    from fractions import Fraction
+    T, E, H = 3, 4, 264
+    rng = np.random.default_rng(22)
+    x = _bf16(rng.standard_normal((T, H)))
+    wg = _bf16(rng.standard_normal((E, H)) * 0.02)
+    lg = orc.router_logits(x, wg)
+    xf, wf = syn.bf16_bits_to_f32(x).astype(np.float64), syn.bf16_bits_to_f32(wg).astype(np.float64)
+    for t in range(T):
+        for e in range(E):
+            exact = sum((Fraction(float(a)) * Fraction(float(b)) for a, b in zip(xf[t], wf[e])), Fraction(0))
+            mag = float(np.sum(np.abs(xf[t] * wf[e])))
+            err = abs(Fraction(float(lg[t, e])) - exact)
+            ulp = float(np.spacing(np.float32(max(abs(float(exact)), abs(float(lg[t, e]))))))
+            assert err <= Fraction(0.5 * ulp) + Fraction((H + 8) * 2.0 ** -53 * mag)
+
+
+@pytest.mark.parametrize("hs,expect", [
+    ((0, 256, 512), 0.0),     # one lane, ascending h: 2^60 + 1 loses the 1
+    ((0, 8, 16), 1.0),        # lanes 0, 1, 2: (s0 + s2) + (s1 + s3) keeps it
+    ((0, 8, 128), 1.0),       # lanes 0, 1, 16: (s0 + s16) + s1 keeps it
+])
+def test_router_logits_follow_the_fixed_order(hs, expect):
+    """Products 2^60, 1, -2^60 at chosen positions: the result depends on the
+    association, which pins the lane assignment and the xor tree."""
+    H = 640
+    x = np.zeros((1, H), dtype=np.float32)
+    w = np.zeros((1, H), dtype=np.float32)
+    x[0, hs[0]], w[0, hs[0]] = 2.0 ** 30, 2.0 ** 30
+    x[0, hs[1]], w[0, hs[1]] = 1.0, 1.0
+    x[0, hs[2]], w[0, hs[2]] = -(2.0 ** 30), 2.0 ** 30
+    assert orc.router_logits(_bf16(x), _bf16(w))[0, 0] == np.float32(expect)
+
+
+def test_router_logits_feed_routing_like_given_logits():
+    """The synthetic router-logit recipe and the oracle's router agree to fp32
+    rounding on the seeded Mixtral-shaped tokens, and route identically."""
+    wl = syn.WORKLOADS["mixtral_decode"].with_T(16)
+    x = syn.tokens(wl)
+    lg = orc.router_logits(x, syn.router_weight(wl))
+    ref = syn.router_logits(wl, x)
+    assert np.allclose(lg, ref, rtol=1e-6, atol=1e-7)
+    assert np.array_equal(orc.route(lg, k=2)[0], orc.route(ref, k=2)[0])
