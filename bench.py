@@ -352,6 +352,25 @@ def ours_main(args, wl):
     torch.cuda.synchronize(dev)
     t_g1 = statistics.mean(g1[2 * j].elapsed_time(g1[2 * j + 1]) for j in range(args.steps))
     t_g2 = statistics.mean(g2[2 * j].elapsed_time(g2[2 * j + 1]) for j in range(args.steps))
+
+    # the optional router step (logits = x . W_g^T and top-k in one launch),
+    # for workloads whose logits come from a router weight
+    router = None
+    if wl.logits == "router":
+        wg = to_dev(syn.router_weight(wl))
+        rl = torch.empty((wl.T, wl.E), dtype=torch.float32, device=dev)
+        rids = torch.empty((wl.T, wl.k), dtype=torch.int32, device=dev)
+        rw = torch.empty((wl.T, wl.k), dtype=torch.float32, device=dev)
+        moe.router_topk(shape, x, wg, rl, rids, rw, ws, stream)
+        r0, r1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        r0.record(stream)
+        for _ in range(args.steps):
+            moe.router_topk(shape, x, wg, rl, rids, rw, ws, stream)
+        r1.record(stream)
+        torch.cuda.synchronize(dev)
+        t_r = r0.elapsed_time(r1) / args.steps
+        router = {"kernel": "router_topk (x . W_g^T in fp64, fixed order, + top-k)", "ms": t_r,
+                  "bytes": wl.T * wl.H * 2 + wl.E * wl.H * 2 + wl.T * wl.E * 4 + wl.T * wl.k * 8}
     w13_bytes = active * 2 * wl.H * wl.I * esz
     w2_bytes = active * wl.H * wl.I * esz
     aesz = 1 if wl.adtype else 2
@@ -455,6 +474,7 @@ def ours_main(args, wl):
                 "overlap": "double-buffered: H2D and D2H on their own copy streams overlap the layer of "
                            "the neighbouring step; the host reads every step's result"},
         "gpu_launches": launches_per_step * args.steps,
+        "router": router,
         "clocks": clk,
     }
     if rank == 0 and world == 1 and not args.no_cpu:

@@ -125,6 +125,24 @@ int moe_route_topk(const moe_shape_t *shape, const float *logits, int32_t *ids, 
                    moe_stream_t stream);
 
 /*
+ * Step 0+1 - router logits and top-k in one launch (the Chinese retelling,
+ * section "2. 用于FP8量化的Triton后端路由": routing is decided inside the
+ * fused kernel, without host control flow).
+ *   x [T, H] bf16 and wg [E, H] bf16 (the router weight) in, both 16-byte
+ *   aligned; logits [T, E] fp32, ids [T, k] and w [T, k] out, ids and w as
+ *   for moe_route_topk on those logits.
+ *   logits[t,e] = sum_h x[t,h] * wg[e,h] in a fixed order, so that routing is
+ *   reproducible bit for bit: in double precision, 32 partial sums where sum
+ *   l takes, in ascending h, the 8-element chunks h/8 congruent to l mod 32;
+ *   then s_l += s_(l xor o) for o = 16, 8, 4, 2, 1; one rounding to fp32.
+ *   ws: workspace of moe_workspace_size bytes (per-token tickets).
+ * Errors: MOE_ERR_INVALID_ARG for NULL or misaligned pointers,
+ * MOE_ERR_WORKSPACE_TOO_SMALL.
+ */
+int moe_router_topk(const moe_shape_t *shape, const void *x, const void *wg, float *logits, int32_t *ids,
+                    float *w, void *ws, size_t ws_bytes, moe_stream_t stream);
+
+/*
  * Step 2 - alignment / permutation ("data shuffling").
  *   ids [T, k] int32 in (each in 0..E-1).  Out:
  *     counts      [E + n_shared]   rows of each expert (T for shared experts)
@@ -231,6 +249,16 @@ int moe_fused_forward(const moe_shape_t *shape, const void *x, const float *logi
                       const void *w13, const float *w13_scale, const void *w2,
                       const float *w2_scale, float a1_scale, float a2_scale, void *out,
                       void *ws, size_t ws_bytes, moe_stream_t stream);
+
+/*
+ * The same layer starting from the router weight: step 0+1
+ * (moe_router_topk, logits kept in the workspace) instead of step 1.
+ * wg [E, H] bf16, 16-byte aligned; everything else as moe_fused_forward.
+ */
+int moe_fused_forward_router(const moe_shape_t *shape, const void *x, const void *wg, const void *w13,
+                             const float *w13_scale, const void *w2, const float *w2_scale,
+                             float a1_scale, float a2_scale, void *out, void *ws, size_t ws_bytes,
+                             moe_stream_t stream);
 
 /*
  * Device status written by the kernels into `ws`: copies it to *status

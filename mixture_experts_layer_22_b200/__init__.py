@@ -29,7 +29,8 @@ STATUS = {0: "MOE_OK", -1: "MOE_ERR_INVALID_ARG", -2: "MOE_ERR_UNSUPPORTED",
 EXPORTS = ["moe_max_rows", "moe_workspace_size", "moe_route_topk", "moe_align_permute", "moe_gather",
            "moe_grouped_gemm_swiglu", "moe_grouped_gemm_down", "moe_combine", "moe_fused_forward",
            "moe_get_device_status", "moe_reset_device_status", "moe_status_string",
-           "moe_last_launch_count", "moe_align_permute_noalloc"]
+           "moe_last_launch_count", "moe_align_permute_noalloc", "moe_router_topk",
+           "moe_fused_forward_router"]
 
 
 class MoeError(RuntimeError):
@@ -79,6 +80,8 @@ def lib() -> C.CDLL:
             "moe_status_string": [C.c_int],
             "moe_last_launch_count": [],
             "moe_align_permute_noalloc": [S, P, P, P, P, P, P, P],
+            "moe_router_topk": [S, P, P, P, P, P, P, C.c_size_t, P],
+            "moe_fused_forward_router": [S, P, P, P, P, P, P, C.c_float, C.c_float, P, P, C.c_size_t, P],
         }
         for name, args in sig.items():
             fn = getattr(L, name)
@@ -143,6 +146,12 @@ def route_topk(shape, logits, ids, w, stream=None):
            "moe_route_topk")
 
 
+def router_topk(shape, x, wg, logits, ids, w, ws, stream=None):
+    """Router logits x . wg^T (fixed summation order) and top-k in one launch."""
+    _check(lib().moe_router_topk(C.byref(shape), _ptr(x), _ptr(wg), _ptr(logits), _ptr(ids), _ptr(w),
+                                 _ptr(ws), ws.numel(), _stream(stream)), "moe_router_topk")
+
+
 def align_permute(shape, ids, counts, offsets, sorted_rows, inv, ws, stream=None):
     _check(lib().moe_align_permute(C.byref(shape), _ptr(ids), _ptr(counts), _ptr(offsets),
                                    _ptr(sorted_rows), _ptr(inv), _ptr(ws), ws.numel(), _stream(stream)),
@@ -184,6 +193,12 @@ def fused_forward(shape, x, logits, w13, w13_scale, w2, w2_scale, a1, a2, out, w
     _check(lib().moe_fused_forward(C.byref(shape), _ptr(x), _ptr(logits), _ptr(w13), _ptr(w13_scale),
                                    _ptr(w2), _ptr(w2_scale), a1, a2, _ptr(out), _ptr(ws), ws.numel(),
                                    _stream(stream)), "moe_fused_forward")
+
+
+def fused_forward_router(shape, x, wg, w13, w13_scale, w2, w2_scale, a1, a2, out, ws, stream=None):
+    _check(lib().moe_fused_forward_router(C.byref(shape), _ptr(x), _ptr(wg), _ptr(w13), _ptr(w13_scale),
+                                          _ptr(w2), _ptr(w2_scale), a1, a2, _ptr(out), _ptr(ws), ws.numel(),
+                                          _stream(stream)), "moe_fused_forward_router")
 
 
 def device_status(ws, stream=None) -> int:

@@ -60,6 +60,7 @@ cudaError_t launch_kernel(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t 
 struct WsLayout {
     size_t ctrl, ids, w, counts, offsets, chunk_hist, chunk_base, sorted_rows, inv;
     size_t xp, h, y, counters, partials;
+    size_t tickets, logits;   // router: per-token tickets (zeroed with the control words), logits
     size_t total;
     int64_t max_rows;
     int n_chunks;
@@ -80,6 +81,9 @@ int validate_shape(const moe_shape_t *s, bool need_gemm);
 // ---- launchers (return cudaError_t of the launch) ----
 cudaError_t launch_route(const moe_shape_t &s, const float *logits, int32_t *ids, float *w,
                          cudaStream_t st);
+// router logits x . Wg^T and top-k in one launch; tickets [T] must be zero
+cudaError_t launch_router(const moe_shape_t &s, const void *x, const void *wg, float *logits,
+                          int32_t *tickets, int32_t *ids, float *w, cudaStream_t st, bool chained);
 // `chained`: launched by moe_fused_forward after its first kernel (PDL
 // launch; the control words and GEMM tile counters were zeroed at the start
 // of the call)

@@ -72,6 +72,9 @@ bool ws_layout(const moe_shape_t &s, WsLayout &L)
     // stream-K tile counters right after the control words (one memset
     // clears both): GEMM1 uses the first half, GEMM2 the second
     L.counters = o;    o += up256(4 * kMaxCtas * 4);
+    // router tickets, also cleared by that memset
+    L.tickets = o;     o += up256(static_cast<size_t>(s.T) * 4);
+    L.logits = o;      o += up256(static_cast<size_t>(s.T) * s.E * 4);
     L.ids = o;         o += up256(R * 4);
     L.w = o;           o += up256(R * 4);
     L.counts = o;      o += up256(Et * 4);
@@ -256,7 +259,27 @@ int moe_combine(const moe_shape_t *shape, const float *y, const float *w, const 
     return cuda_status(launch_combine(*shape, y, w, inv, offsets, out, reinterpret_cast<cudaStream_t>(stream)));
 }
 
-int moe_fused_forward(const moe_shape_t *shape, const void *x, const float *logits,
+int moe_router_topk(const moe_shape_t *shape, const void *x, const void *wg, float *logits, int32_t *ids,
+                    float *w, void *ws, size_t ws_bytes, moe_stream_t stream)
+{
+    g_launches = 0;
+    int st = validate_shape(shape, false);
+    if (st != MOE_OK) return st;
+    if (!x || !wg || !logits || !ids || !w || !ws) return MOE_ERR_INVALID_ARG;
+    if (!aligned(x, 16) || !aligned(wg, 16) || !aligned(ws, 256)) return MOE_ERR_INVALID_ARG;
+    WsLayout L;
+    ws_layout(*shape, L);
+    if (ws_bytes < L.total) return MOE_ERR_WORKSPACE_TOO_SMALL;
+    cudaStream_t sm = reinterpret_cast<cudaStream_t>(stream);
+    int32_t *tickets = reinterpret_cast<int32_t *>(static_cast<char *>(ws) + L.tickets);
+    if (cudaMemsetAsync(tickets, 0, static_cast<size_t>(shape->T) * sizeof(int32_t), sm) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    g_launches = 1;
+    return cuda_status(launch_router(*shape, x, wg, logits, tickets, ids, w, sm, false));
+}
+
+// The fused layer from router logits (wg == NULL) or from the router weight.
+static int fused_impl(const moe_shape_t *shape, const void *x, const float *logits, const void *wg,
                       const void *w13, const float *w13_scale, const void *w2,
                       const float *w2_scale, float a1_scale, float a2_scale, void *out, void *ws,
                       size_t ws_bytes, moe_stream_t stream)
@@ -264,9 +287,10 @@ int moe_fused_forward(const moe_shape_t *shape, const void *x, const float *logi
     g_launches = 0;
     int st = validate_shape(shape, true);
     if (st != MOE_OK) return st;
-    if (!x || !logits || !w13 || !w2 || !out || !ws) return MOE_ERR_INVALID_ARG;
+    if (!x || (!logits && !wg) || !w13 || !w2 || !out || !ws) return MOE_ERR_INVALID_ARG;
     if (!aligned(x, 16) || !aligned(out, 16) || !aligned(w13, 16) || !aligned(w2, 16) || !aligned(ws, 256))
         return MOE_ERR_INVALID_ARG;
+    if (wg && !aligned(wg, 16)) return MOE_ERR_INVALID_ARG;
     if (shape->wdtype == MOE_E4M3 && (!w13_scale || !w2_scale)) return MOE_ERR_INVALID_ARG;
     if (shape->adtype == MOE_E4M3 && (!(a1_scale > 0.0f) || !(a2_scale > 0.0f))) return MOE_ERR_INVALID_ARG;
     const moe_shape_t &s = *shape;
@@ -286,12 +310,17 @@ int moe_fused_forward(const moe_shape_t *shape, const void *x, const float *logi
     void *h = b + L.h;
     float *y = reinterpret_cast<float *>(b + L.y);
 
-    // One memset clears the status, the align ticket and both GEMMs' tile
-    // counters.  Every later kernel is a programmatic dependent launch of the
-    // one before it, so there is no other non-kernel node in the sequence.
-    cudaError_t e = cudaMemsetAsync(ctrl, 0, L.counters + 4 * kMaxCtas * sizeof(int32_t) - L.ctrl, sm);
+    // One memset clears the status, the align ticket, both GEMMs' tile
+    // counters and the router's tickets (adjacent in the workspace).  Every
+    // later kernel is a programmatic dependent launch of the one before it,
+    // so there is no other non-kernel node in the sequence.
+    cudaError_t e = cudaMemsetAsync(ctrl, 0, L.tickets + static_cast<size_t>(s.T) * sizeof(int32_t) - L.ctrl, sm);
     if (e != cudaSuccess) return MOE_ERR_CUDA;
-    e = launch_route(s, logits, ids, w, sm);
+    if (wg)
+        e = launch_router(s, x, wg, reinterpret_cast<float *>(b + L.logits),
+                          reinterpret_cast<int32_t *>(b + L.tickets), ids, w, sm, false);
+    else
+        e = launch_route(s, logits, ids, w, sm);
     if (e != cudaSuccess) return MOE_ERR_CUDA;
     g_launches += 1;
     e = launch_align(s, ids, counts, offsets, rows, inv, reinterpret_cast<int32_t *>(b + L.chunk_hist),
@@ -335,6 +364,31 @@ int moe_fused_forward(const moe_shape_t *shape, const void *x, const float *logi
     if (e != cudaSuccess) return MOE_ERR_CUDA;
     g_launches += 1;
     return MOE_OK;
+}
+
+int moe_fused_forward(const moe_shape_t *shape, const void *x, const float *logits,
+                      const void *w13, const float *w13_scale, const void *w2,
+                      const float *w2_scale, float a1_scale, float a2_scale, void *out, void *ws,
+                      size_t ws_bytes, moe_stream_t stream)
+{
+    if (!logits) {
+        g_launches = 0;
+        return MOE_ERR_INVALID_ARG;
+    }
+    return fused_impl(shape, x, logits, nullptr, w13, w13_scale, w2, w2_scale, a1_scale, a2_scale, out, ws,
+                      ws_bytes, stream);
+}
+
+int moe_fused_forward_router(const moe_shape_t *shape, const void *x, const void *wg, const void *w13,
+                             const float *w13_scale, const void *w2, const float *w2_scale, float a1_scale,
+                             float a2_scale, void *out, void *ws, size_t ws_bytes, moe_stream_t stream)
+{
+    if (!wg) {
+        g_launches = 0;
+        return MOE_ERR_INVALID_ARG;
+    }
+    return fused_impl(shape, x, nullptr, wg, w13, w13_scale, w2, w2_scale, a1_scale, a2_scale, out, ws,
+                      ws_bytes, stream);
 }
 
 int moe_get_device_status(const void *ws, int32_t *status, moe_stream_t stream)

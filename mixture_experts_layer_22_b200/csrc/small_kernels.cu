@@ -39,21 +39,13 @@ __device__ __forceinline__ float warp_max(float v)
     return v;
 }
 
-// One warp per token.  Lane l holds logits l, l+32, ...; the k winners are
-// found by k rounds of a warp-wide arg-max over the 64-bit key
+// Top-k of one token by one warp.  Lane l holds logits l, l+32, ...; the k
+// winners are found by k rounds of a warp-wide arg-max over the 64-bit key
 // (logit key, ~expert id): larger logit first, ties to the lower id.
 template <int kSlots>
-__global__ void __launch_bounds__(256) route_topk_kernel(const float *__restrict__ logits, int T,
-                                                         int E, int k, int gate, int renorm,
-                                                         float routed_scale, int32_t *ids,
-                                                         float *w)
+__device__ __forceinline__ void route_warp(const float *l, int E, int k, int gate, int renorm,
+                                           float routed_scale, int32_t *ids_t, float *w_t, int lane)
 {
-    grid_dep_wait();
-    grid_dep_launch();
-    const int lane = threadIdx.x & 31;
-    const int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-    if (t >= T) return;
-    const float *l = logits + static_cast<size_t>(t) * E;
     uint64_t key[kSlots];
     uint32_t taken = 0;
 #pragma unroll
@@ -103,9 +95,25 @@ __global__ void __launch_bounds__(256) route_topk_kernel(const float *__restrict
         wt = renorm ? s / warp_sum(s) : s;
     }
     if (mine) {
-        ids[static_cast<size_t>(t) * k + lane] = my_id;
-        w[static_cast<size_t>(t) * k + lane] = wt * routed_scale;
+        ids_t[lane] = my_id;
+        w_t[lane] = wt * routed_scale;
     }
+}
+
+// One warp per token.
+template <int kSlots>
+__global__ void __launch_bounds__(256) route_topk_kernel(const float *__restrict__ logits, int T,
+                                                         int E, int k, int gate, int renorm,
+                                                         float routed_scale, int32_t *ids,
+                                                         float *w)
+{
+    grid_dep_wait();
+    grid_dep_launch();
+    const int lane = threadIdx.x & 31;
+    const int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    if (t >= T) return;
+    route_warp<kSlots>(logits + static_cast<size_t>(t) * E, E, k, gate, renorm, routed_scale,
+                       ids + static_cast<size_t>(t) * k, w + static_cast<size_t>(t) * k, lane);
 }
 
 cudaError_t launch_route(const moe_shape_t &s, const float *logits, int32_t *ids, float *w,
@@ -123,6 +131,85 @@ cudaError_t launch_route(const moe_shape_t &s, const float *logits, int32_t *ids
     else MOE_ROUTE(16);
 #undef MOE_ROUTE
     return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------ router
+// Router logits and top-k in one launch (the step before routing; the Chinese
+// retelling, section "2. 用于FP8量化的Triton后端路由", keeps routing inside
+// the fused kernel).  l[t,e] = sum_h x[t,h] * Wg[e,h] in a fixed order, so
+// that the result does not depend on the launch shape:
+//   lane l of a warp sums in double, in ascending h, the products of the
+//   8-element chunks c (16-byte loads) with c mod 32 == l; the warp combines
+//   its 32 partial sums by s_l += s_(l xor o), o = 16, 8, 4, 2, 1; the sum is
+//   rounded once to fp32.
+// Block (t, g) computes token t's logits of experts [32 g, 32 g + 32), one
+// warp per expert at a time.  The last block of token t to finish (ticket)
+// selects its top-k from all E logits, as route_topk_kernel does.
+__device__ __forceinline__ double dot8(uint4 a, uint4 b, double acc)
+{
+    const uint32_t wa[4] = {a.x, a.y, a.z, a.w}, wb[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        acc = fma(static_cast<double>(__uint_as_float(wa[i] << 16)),
+                  static_cast<double>(__uint_as_float(wb[i] << 16)), acc);      // exact product
+        acc = fma(static_cast<double>(__uint_as_float(wa[i] & 0xFFFF0000u)),
+                  static_cast<double>(__uint_as_float(wb[i] & 0xFFFF0000u)), acc);
+    }
+    return acc;
+}
+
+template <int kSlots>
+__global__ void __launch_bounds__(256) router_topk_kernel(const uint4 *__restrict__ x, const uint4 *__restrict__ wg,
+                                                          int H, int E, int k, int gate, int renorm,
+                                                          float routed_scale, float *logits, int32_t *tickets,
+                                                          int32_t *ids, float *w)
+{
+    grid_dep_wait();
+    grid_dep_launch();
+    __shared__ float s_l[kMaxExperts];
+    __shared__ int s_last;
+    const int t = blockIdx.x, g = blockIdx.y;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int nc = H / 8;
+    const uint4 *xr = x + static_cast<size_t>(t) * nc;
+    for (int j = warp; j < 32; j += 8) {
+        const int e = g * 32 + j;
+        if (e >= E) break;
+        const uint4 *wr = wg + static_cast<size_t>(e) * nc;
+        double acc = 0.0;
+        for (int c = lane; c < nc; c += 32) acc = dot8(__ldg(xr + c), __ldg(wr + c), acc);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+        if (lane == 0) logits[static_cast<size_t>(t) * E + e] = __double2float_rn(acc);
+    }
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) s_last = atomicAdd(&tickets[t], 1) == static_cast<int>(gridDim.y) - 1;
+    __syncthreads();
+    if (!s_last) return;
+    __threadfence();
+    for (int e = threadIdx.x; e < E; e += blockDim.x) s_l[e] = __ldcg(&logits[static_cast<size_t>(t) * E + e]);
+    __syncthreads();
+    if (warp == 0)
+        route_warp<kSlots>(s_l, E, k, gate, renorm, routed_scale, ids + static_cast<size_t>(t) * k,
+                           w + static_cast<size_t>(t) * k, lane);
+}
+
+cudaError_t launch_router(const moe_shape_t &s, const void *x, const void *wg, float *logits,
+                          int32_t *tickets, int32_t *ids, float *w, cudaStream_t st, bool chained)
+{
+    const dim3 grid(s.T, (s.E + 31) / 32);
+    const int slots = (s.E + 31) / 32;
+    const uint4 *xv = static_cast<const uint4 *>(x), *wv = static_cast<const uint4 *>(wg);
+#define MOE_ROUTER(N)                                                                                  \
+    return launch_kernel(router_topk_kernel<N>, grid, dim3(256), 0, st, chained, xv, wv, s.H, s.E, s.k, \
+                         s.gate, s.renorm, s.routed_scale, logits, tickets, ids, w)
+    if (slots <= 1) MOE_ROUTER(1);
+    if (slots <= 2) MOE_ROUTER(2);
+    if (slots <= 4) MOE_ROUTER(4);
+    if (slots <= 8) MOE_ROUTER(8);
+    MOE_ROUTER(16);
+#undef MOE_ROUTER
 }
 
 // ------------------------------------------------------------------ align

@@ -84,6 +84,18 @@ def test_null_pointers_rejected_before_launch(lib):
     assert lib.moe_align_permute(None, None, None, None, None, None, None, 0, None) == -1
 
 
+def test_router_entry_points_reject_bad_arguments(lib):
+    s = _shape(H=256, I=256)
+    need = moe.workspace_size(s)
+    assert lib.moe_router_topk(C.byref(s), None, 256, 256, 256, 256, 256, need, None) == -1
+    assert lib.moe_router_topk(C.byref(s), 264, 256, 256, 256, 256, 256, need, None) == -1   # misaligned x
+    assert lib.moe_router_topk(C.byref(s), 256, 256, 256, 256, 256, 256, need - 1, None) == -3
+    assert lib.moe_fused_forward_router(C.byref(s), 256, None, 256, None, 256, None, 1.0, 1.0, 256, 256, need,
+                                        None) == -1
+    assert lib.moe_fused_forward_router(C.byref(s), 256, 264, 256, None, 256, None, 1.0, 1.0, 256, 256, need,
+                                        None) == -1
+
+
 def test_workspace_too_small_rejected(lib):
     s = _shape()
     need = moe.workspace_size(s)

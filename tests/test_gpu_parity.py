@@ -403,3 +403,53 @@ def test_e4m3_weight_expansion_is_exact(mode):
         assert rel_err(outs[0], outs[1], "bf16") <= 1e-3
     else:
         assert rel_err(outs[0], outs[1]) <= 1e-5
+
+
+# ------------------------------------------------------------------ router (step 0+1)
+ROUTER_CASES = [W["tiny"], W["mixtral_decode"],
+                dataclasses.replace(W["dsv3_decode_fp8w"], wdtype=syn.BF16),
+                syn.Workload("router_odd", T=77, H=136, I=128, E=45, k=3, seed=12)]
+
+
+@pytest.mark.parametrize("wl", ROUTER_CASES, ids=lambda w: w.name)
+def test_router_topk_bit_exact(wl):
+    """Router logits bit for bit against the oracle's fixed-order sum, then
+    ids bit-exact and weights within 2e-6 of the oracle's routing of those
+    logits."""
+    x = syn.tokens(wl)
+    wg = syn.router_weight(wl)
+    ref_l = orc.router_logits(x, wg)
+    ref_ids, ref_w = orc.route(ref_l, k=wl.k, gate=wl.gate, renorm=wl.renorm, routed_scale=wl.routed_scale)
+    s = _shape(wl)
+    ws = moe.workspace(s)
+    lg = torch.full((wl.T, wl.E), float("nan"), dtype=torch.float32, device="cuda")
+    ids = torch.empty((wl.T, wl.k), dtype=torch.int32, device="cuda")
+    w = torch.empty((wl.T, wl.k), dtype=torch.float32, device="cuda")
+    for _ in range(2):                                # a rerun reuses the workspace tickets
+        moe.router_topk(s, dev_bf16(x), dev_bf16(wg), lg, ids, w, ws)
+        torch.cuda.synchronize()
+        assert np.array_equal(lg.cpu().numpy().view(np.uint32), ref_l.view(np.uint32))
+        assert np.array_equal(ids.cpu().numpy(), ref_ids)
+        assert np.allclose(w.cpu().numpy(), ref_w, rtol=2e-6, atol=1e-7)
+
+
+@pytest.mark.parametrize("wl", [W["tiny"], W["mixtral_decode"].with_T(8),
+                                W["dsv3_decode_fp8w"].with_T(8)], ids=lambda w: f"{w.name}_T{w.T}")
+def test_fused_forward_router_equals_logits_path(wl):
+    """The layer started from the router weight equals, bit for bit, the layer
+    given the oracle's router logits, and matches the oracle's layer."""
+    d = syn.make_inputs(wl)
+    wg = syn.router_weight(wl)
+    d["logits"] = orc.router_logits(d["x"], wg)
+    L = Layer(wl, d)
+    via_logits = L.run()
+    moe.reset_device_status(L.ws)
+    out = torch.empty_like(L.out)
+    moe.fused_forward_router(L.shape, L.x, dev_bf16(wg), L.w13, L.s13, L.w2, L.s2, L.a1, L.a2, out, L.ws)
+    torch.cuda.synchronize()
+    assert L.status() == 0
+    via_router = bf16_to_f64(host_bf16_bits(out))
+    assert np.array_equal(via_router, via_logits)
+    toks = np.unique(np.linspace(0, wl.T - 1, min(wl.T, 6)).astype(np.int32))
+    ref = oracle_forward(wl, d, tokens=toks)
+    assert rel_err(via_router[toks], ref, "bf16") <= BF16_TOL
