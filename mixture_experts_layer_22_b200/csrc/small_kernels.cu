@@ -142,9 +142,11 @@ cudaError_t launch_route(const moe_shape_t &s, const float *logits, int32_t *ids
 //   8-element chunks c (16-byte loads) with c mod 32 == l; the warp combines
 //   its 32 partial sums by s_l += s_(l xor o), o = 16, 8, 4, 2, 1; the sum is
 //   rounded once to fp32.
-// Block (t, g) computes token t's logits of experts [32 g, 32 g + 32), one
-// warp per expert at a time.  The last block of token t to finish (ticket)
-// selects its top-k from all E logits, as route_topk_kernel does.
+// Block (t, g) computes token t's logits of experts [32 g, 32 g + 32): warp
+// w takes experts 32 g + 4 w .. 32 g + 4 w + 3 together (four independent
+// accumulation chains per lane, one load of x for four rows of Wg; the order
+// within each chain is the one above).  The last block of token t to finish
+// (ticket) selects its top-k from all E logits, as route_topk_kernel does.
 __device__ __forceinline__ double dot8(uint4 a, uint4 b, double acc)
 {
     const uint32_t wa[4] = {a.x, a.y, a.z, a.w}, wb[4] = {b.x, b.y, b.z, b.w};
@@ -172,15 +174,27 @@ __global__ void __launch_bounds__(256) router_topk_kernel(const uint4 *__restric
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int nc = H / 8;
     const uint4 *xr = x + static_cast<size_t>(t) * nc;
-    for (int j = warp; j < 32; j += 8) {
-        const int e = g * 32 + j;
-        if (e >= E) break;
-        const uint4 *wr = wg + static_cast<size_t>(e) * nc;
-        double acc = 0.0;
-        for (int c = lane; c < nc; c += 32) acc = dot8(__ldg(xr + c), __ldg(wr + c), acc);
+    constexpr int kPer = 4;                      // experts per warp
+    const int e0 = g * 32 + warp * kPer;
+    if (e0 < E) {
+        const uint4 *wr[kPer];
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-        if (lane == 0) logits[static_cast<size_t>(t) * E + e] = __double2float_rn(acc);
+        for (int q = 0; q < kPer; ++q)             // rows past E repeat the last one (not stored)
+            wr[q] = wg + static_cast<size_t>(min(e0 + q, E - 1)) * nc;
+        double acc[kPer];
+#pragma unroll
+        for (int q = 0; q < kPer; ++q) acc[q] = 0.0;
+        for (int c = lane; c < nc; c += 32) {
+            const uint4 a = __ldg(xr + c);
+#pragma unroll
+            for (int q = 0; q < kPer; ++q) acc[q] = dot8(a, __ldg(wr[q] + c), acc[q]);
+        }
+#pragma unroll
+        for (int q = 0; q < kPer; ++q) {
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) acc[q] += __shfl_xor_sync(0xffffffffu, acc[q], o);
+            if (lane == 0 && e0 + q < E) logits[static_cast<size_t>(t) * E + e0 + q] = __double2float_rn(acc[q]);
+        }
     }
     __threadfence();
     __syncthreads();
