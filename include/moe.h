@@ -261,6 +261,17 @@ int moe_fused_forward_router(const moe_shape_t *shape, const void *x, const void
                              moe_stream_t stream);
 
 /*
+ * Self-test of the failure path (no counterpart on the pages): launches one
+ * block whose two bounded pipeline waits run out, because nothing arrives on
+ * their barriers.  The first gives up after the library's wait limit (2 s),
+ * raises the block's abort flag, and the second then gives up at once.  The
+ * block writes MOE_ERR_TIMEOUT to the status word at the start of `ws` and
+ * exits, so the CUDA context stays usable.  gave_up (device int32) receives
+ * the number of waits that gave up (2).  Asynchronous on `stream`.
+ */
+int moe_selftest_wait_timeout(void *ws, int32_t *gave_up, moe_stream_t stream);
+
+/*
  * Device status written by the kernels into `ws`: copies it to *status
  * (host) after synchronising `stream` -- the one call here that waits.
  * MOE_OK when no kernel reported a problem since the last reset.

@@ -30,7 +30,7 @@ EXPORTS = ["moe_max_rows", "moe_workspace_size", "moe_route_topk", "moe_align_pe
            "moe_grouped_gemm_swiglu", "moe_grouped_gemm_down", "moe_combine", "moe_fused_forward",
            "moe_get_device_status", "moe_reset_device_status", "moe_status_string",
            "moe_last_launch_count", "moe_align_permute_noalloc", "moe_router_topk",
-           "moe_fused_forward_router"]
+           "moe_fused_forward_router", "moe_selftest_wait_timeout"]
 
 
 class MoeError(RuntimeError):
@@ -82,6 +82,7 @@ def lib() -> C.CDLL:
             "moe_align_permute_noalloc": [S, P, P, P, P, P, P, P],
             "moe_router_topk": [S, P, P, P, P, P, P, C.c_size_t, P],
             "moe_fused_forward_router": [S, P, P, P, P, P, P, C.c_float, C.c_float, P, P, C.c_size_t, P],
+            "moe_selftest_wait_timeout": [P, P, P],
         }
         for name, args in sig.items():
             fn = getattr(L, name)
@@ -199,6 +200,12 @@ def fused_forward_router(shape, x, wg, w13, w13_scale, w2, w2_scale, a1, a2, out
     _check(lib().moe_fused_forward_router(C.byref(shape), _ptr(x), _ptr(wg), _ptr(w13), _ptr(w13_scale),
                                           _ptr(w2), _ptr(w2_scale), a1, a2, _ptr(out), _ptr(ws), ws.numel(),
                                           _stream(stream)), "moe_fused_forward_router")
+
+
+def selftest_wait_timeout(ws, gave_up, stream=None):
+    """Launch the failure-path self-test (about 2 s on the GPU): its bounded
+    waits run out and it reports MOE_ERR_TIMEOUT in ws's status word."""
+    _check(lib().moe_selftest_wait_timeout(_ptr(ws), _ptr(gave_up), _stream(stream)), "moe_selftest_wait_timeout")
 
 
 def device_status(ws, stream=None) -> int:

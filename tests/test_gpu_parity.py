@@ -453,3 +453,27 @@ def test_fused_forward_router_equals_logits_path(wl):
     toks = np.unique(np.linspace(0, wl.T - 1, min(wl.T, 6)).astype(np.int32))
     ref = oracle_forward(wl, d, tokens=toks)
     assert rel_err(via_router[toks], ref, "bf16") <= BF16_TOL
+
+
+# ------------------------------------------------------------------ failure path
+def test_bounded_wait_times_out_and_context_stays_usable():
+    """A pipeline wait on a barrier that nothing arrives on gives up after the
+    wait limit, the abort flag stops the block's other wait, the status word
+    reads MOE_ERR_TIMEOUT, and the next layer call on the same context runs
+    correctly."""
+    import time
+    wl = W["tiny"]
+    d = syn.make_inputs(wl)
+    L = Layer(wl, d)
+    moe.reset_device_status(L.ws)
+    gave_up = torch.full((1,), -1, dtype=torch.int32, device="cuda")
+    t0 = time.perf_counter()
+    moe.selftest_wait_timeout(L.ws, gave_up)
+    torch.cuda.synchronize()
+    dt = time.perf_counter() - t0
+    assert moe.device_status(L.ws) == -6
+    assert int(gave_up.item()) == 2
+    assert 1.5 < dt < 30.0
+    got = L.run()                      # resets the status, runs the layer
+    assert L.status() == 0
+    assert rel_err(got, oracle_forward(wl, d), "bf16") <= BF16_TOL
