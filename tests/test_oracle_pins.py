@@ -371,3 +371,39 @@ def test_router_logits_feed_routing_like_given_logits():
     ref = syn.router_logits(wl, x)
     assert np.allclose(lg, ref, rtol=1e-6, atol=1e-7)
     assert np.array_equal(orc.route(lg, k=2)[0], orc.route(ref, k=2)[0])
+
+
+# ------------------------------------------------------------------ hi/lo split (E4M3 weights, bf16 activations)
+def _split_scale(amax: float) -> float:
+    """Smallest power of two s with amax <= 448 s."""
+    if amax == 0.0:
+        return 1.0
+    s = 2.0 ** np.ceil(np.log2(amax / 448.0))
+    while amax > 448.0 * s:          # guard the log2 rounding at exact powers
+        s *= 2.0
+    while amax <= 224.0 * s:
+        s /= 2.0
+    return s
+
+
+def test_hilo_split_of_bf16_rows_is_exact_but_for_tiny_remainders():
+    """The reading behind the E4M3-weight path: a bf16 row v with the power-of-
+    two scale s splits as hi = e4m3(v/s), lo = e4m3(v/s - hi) with
+    s (hi + lo) == v wherever the remainder is at least 2^-6, and within
+    2^-10 s elsewhere (<= 2^-10 s / (224 s) of the row max), across 9 decades."""
+    rng = np.random.default_rng(23)
+    worst = 0.0
+    for _ in range(200):
+        v = orc.bf16_decode(syn.to_bf16_bits((rng.standard_normal(384) * 10.0 ** rng.uniform(-6, 3)).astype(np.float32)))
+        amax = float(np.abs(v).max())
+        s = _split_scale(amax)
+        assert amax <= 448.0 * s and (amax > 224.0 * s or s == 1.0)
+        q = v / s
+        hi = orc.e4m3_decode(orc.e4m3_encode(q))
+        rem = q - hi
+        lo = orc.e4m3_decode(orc.e4m3_encode(rem))
+        err = np.abs(s * (hi + lo) - v)
+        assert np.all(err[np.abs(rem) >= 2.0 ** -6] == 0.0)
+        assert np.all(err <= 2.0 ** -10 * s)
+        worst = max(worst, float(err.max() / amax))
+    assert worst <= 2.0 ** -10 / 224.0
