@@ -1,7 +1,9 @@
 // common.cuh - internal declarations shared by the library's translation units.
 #pragma once
+#include <atomic>
 #include <cstddef>
 #include <cstdint>
+#include <mutex>
 #include <cuda_runtime.h>
 
 #include "moe.h"
@@ -13,6 +15,34 @@ constexpr int kMaxExpertsTotal = kMaxExperts + 1;
 constexpr int kMaxTopK = 32;
 constexpr int kMaxCtas = 160;               // persistent GEMM grid bound (>= SM count)
 constexpr int kAlignChunk = 1024;           // routed rows per align block
+
+// Host-side setup that CUDA keeps per device (function attributes,
+// occupancy): runs f once for each device it is called on, thread-safe.
+class PerDeviceOnce {
+  public:
+    template <class F>
+    void operator()(F &&f)
+    {
+        int d = 0;
+        cudaGetDevice(&d);
+        if (d < 0 || d >= kDevices) {            // beyond the table: always run (idempotent)
+            std::lock_guard<std::mutex> g(m_);
+            f();
+            return;
+        }
+        if (done_[d].load(std::memory_order_acquire)) return;
+        std::lock_guard<std::mutex> g(m_);
+        if (!done_[d].load(std::memory_order_relaxed)) {
+            f();
+            done_[d].store(true, std::memory_order_release);
+        }
+    }
+
+  private:
+    static constexpr int kDevices = 64;
+    std::atomic<bool> done_[kDevices]{};
+    std::mutex m_;
+};
 
 // Control words at the start of the workspace.
 struct Ctrl {

@@ -873,30 +873,37 @@ static bool make_map(CUtensorMap *m, const void *base, bool u8, uint64_t rows, u
     return r == CUDA_SUCCESS;
 }
 
+// SMs of the current device (the persistent grid size), cached per device.
 static int sm_count()
 {
-    static int n = 0;
+    static std::atomic<int> cache[64];
+    int dev = 0;
+    cudaGetDevice(&dev);
+    int n = (dev >= 0 && dev < 64) ? cache[dev].load(std::memory_order_relaxed) : 0;
     if (n == 0) {
-        int dev = 0;
-        cudaGetDevice(&dev);
         cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
         if (n <= 0) n = 148;
         if (n > kMaxCtas) n = kMaxCtas;
+        if (dev >= 0 && dev < 64) cache[dev].store(n, std::memory_order_relaxed);
     }
     return n;
 }
 
-// Persistent grid of CTA pairs for the kPair kernel: as many pairs as can be
-// resident at once (two SMs of one GPC each), at most half the SM count.
-template <typename Kern>
-static int pair_grid(Kern kern, int threads, int smem)
+// Persistent grid of CTA pairs for a kPair kernel on the current device: as
+// many pairs as can be resident at once (two SMs of one GPC each), at most
+// half the SM count.  Cached per kernel configuration and device.
+template <class Cf, typename Kern>
+static int pair_grid(Kern kern)
 {
-    static int grid = 0;
+    static std::atomic<int> cache[64];
+    int dev = 0;
+    cudaGetDevice(&dev);
+    int grid = (dev >= 0 && dev < 64) ? cache[dev].load(std::memory_order_relaxed) : 0;
     if (grid == 0) {
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(2 * (sm_count() / 2));
-        cfg.blockDim = dim3(threads);
-        cfg.dynamicSmemBytes = smem;
+        cfg.blockDim = dim3(Cf::kThreads);
+        cfg.dynamicSmemBytes = Cf::kDynSmem;
         cudaLaunchAttribute attr[1];
         attr[0].id = cudaLaunchAttributeClusterDimension;
         attr[0].val.clusterDim.x = 2;
@@ -910,6 +917,7 @@ static int pair_grid(Kern kern, int threads, int smem)
             clusters = 1;
         }
         grid = 2 * (clusters < sm_count() / 2 ? clusters : sm_count() / 2);
+        if (dev >= 0 && dev < 64) cache[dev].store(grid, std::memory_order_relaxed);
     }
     return grid;
 }
@@ -919,10 +927,8 @@ static cudaError_t run_gemm(const moe_shape_t &s, const GemmArgs &a, cudaStream_
 {
     using Cf = Cfg<kMode, kSwap, kFp8, kBN, kHiLo, kPair>;
     auto kern = grouped_gemm_kernel<kMode, kSwap, kFp8, kBN, kHiLo, kPair>;
-    static std::once_flag once;
-    std::call_once(once, [&] {
-        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cf::kDynSmem);
-    });
+    static PerDeviceOnce attrs;          // function attributes are per device
+    attrs([&] { cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cf::kDynSmem); });
     const int Et = s.E + s.n_shared;
     const bool u8 = kFp8;              // activations are E4M3 codes
     const bool u8w = kFp8;             // weights are E4M3 codes
@@ -965,7 +971,7 @@ static cudaError_t run_gemm(const moe_shape_t &s, const GemmArgs &a, cudaStream_
     }
     if constexpr (kPair) {
         cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = dim3(pair_grid(kern, Cf::kThreads, Cf::kDynSmem));
+        cfg.gridDim = dim3(pair_grid<Cf>(kern));
         cfg.blockDim = dim3(Cf::kThreads);
         cfg.dynamicSmemBytes = Cf::kDynSmem;
         cfg.stream = st;

@@ -440,14 +440,13 @@ cudaError_t launch_align(const moe_shape_t &s, const int32_t *ids, int32_t *coun
 {
     const int R = s.T * s.k, Et = s.E + s.n_shared;
     const int nb = (R + kAlignChunk - 1) / kAlignChunk;
-    static bool attr_done = false;
-    if (!attr_done) {
+    static PerDeviceOnce attrs;
+    attrs([] {
         cudaFuncSetAttribute(align_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              32 * kMaxExpertsTotal * 4);
         cudaFuncSetAttribute(align_single_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              33 * kMaxExpertsTotal * 4);
-        attr_done = true;
-    }
+    });
     if (nb == 1) {
         *launches += 1;
         return launch_kernel(align_single_kernel, dim3(1), dim3(kAlignChunk), 33 * Et * sizeof(int32_t), st,
