@@ -407,3 +407,85 @@ def test_hilo_split_of_bf16_rows_is_exact_but_for_tiny_remainders():
         assert np.all(err <= 2.0 ** -10 * s)
         worst = max(worst, float(err.max() / amax))
     assert worst <= 2.0 ** -10 / 224.0
+
+
+# ------------------------------------------------------------------ E4M3 activations and weights
+# "Tensor-quantised" FP8 (the AWS abstract, backend paragraph; the Russian
+# summary, section "Triton вместо CUTLASS для FP8-квантования"): one fp32
+# scale per expert weight matrix, one static scale per activation tensor,
+# value = code * scale.  These pins rebuild the all-E4M3 layer from pieces
+# that are pinned above (the codec against the format and the library cast,
+# routing against brute force) and numpy matrix products, so that a dropped,
+# doubled or misplaced scale, or a skipped quantisation, fails them.
+def _e4m3_workload(seed=11, n_shared=1):
+    return syn.Workload("t", T=10, H=64, I=48, E=4, k=2, n_shared=n_shared, gate=syn.SIGMOID,
+                        routed_scale=2.5, wdtype=syn.E4M3, adtype=syn.E4M3, seed=seed)
+
+
+def _decoded(codes, scale):
+    return orc.e4m3_decode(codes) * float(scale)
+
+
+def test_fp8_layer_composes_from_pinned_pieces():
+    wl = _e4m3_workload()
+    d = syn.make_inputs(wl)
+    a1 = float(d["a1"])
+    a2 = 0.0153                                   # not a power of two: a scale slip shows
+    E, I = wl.E, wl.I
+    # tokens quantised once with a1 (fp32 quotient), then dequantised
+    xq = orc.quant_e4m3_f32(syn.bf16_bits_to_f32(d["x"]), a1)
+    xd = orc.e4m3_decode(xq) * a1
+    ids, w = orc.route(d["logits"], wl.k, gate=orc.SIGMOID, renorm=True, routed_scale=2.5)
+
+    def mlp(e, xrow):
+        W1 = _decoded(d["w13"][e][:I], d["w13_scale"][e])
+        W3 = _decoded(d["w13"][e][I:], d["w13_scale"][e])
+        W2 = _decoded(d["w2"][e], d["w2_scale"][e])
+        g, u = W1 @ xrow, W3 @ xrow
+        h = g * expit(g) * u
+        hq = orc.e4m3_decode(orc.e4m3_encode(h / a2)) * a2
+        return W2 @ hq
+
+    ref = np.zeros((wl.T, wl.H))
+    for t in range(wl.T):
+        for j in range(wl.k):
+            ref[t] += w[t, j] * mlp(ids[t, j], xd[t])
+        ref[t] += mlp(E, xd[t])                     # the shared expert, weight 1
+    out = orc.forward(d["x"], d["logits"], d["w13"], d["w2"], E=E, k=wl.k, n_shared=1, gate=orc.SIGMOID,
+                      routed_scale=2.5, wdtype=orc.E4M3, adtype=orc.E4M3, w13_scale=d["w13_scale"],
+                      w2_scale=d["w2_scale"], a1=a1, a2=a2)
+    rms = np.sqrt(np.mean(ref ** 2))
+    assert np.max(np.abs(out - ref)) <= 1e-12 * rms
+    # the same layer with the hidden quantisation or the token quantisation
+    # left out is far away: the pin would catch either slip
+    assert np.max(np.abs(orc.forward(d["x"], d["logits"], d["w13"], d["w2"], E=E, k=wl.k, n_shared=1,
+                                     gate=orc.SIGMOID, routed_scale=2.5, wdtype=orc.E4M3, adtype=orc.BF16,
+                                     w13_scale=d["w13_scale"], w2_scale=d["w2_scale"]) - ref)) > 1e-4 * rms
+
+
+def test_fp8_expert_gemm_references_row_by_row():
+    """orc.expert_swiglu / orc.expert_down with E4M3 activations (scales a1,
+    a2) and E4M3 weights with non-unit per-expert scales, against numpy on the
+    decoded values, row by row of every segment (pad rows included)."""
+    wl = _e4m3_workload(seed=12, n_shared=0)
+    d = syn.make_inputs(wl)
+    I, H = wl.I, wl.H
+    offsets = np.array([0, 16, 16, 48, 64], np.int32)          # expert 1 empty
+    rows = int(offsets[-1])
+    a1, a2 = 0.0071, 0.0213
+    xp = syn.random_rows(wl.seed, "xp", rows, H, syn.E4M3)
+    hq = syn.random_rows(wl.seed, "hq", rows, I, syn.E4M3)
+    h = orc.expert_swiglu(xp, offsets, d["w13"], orc.E4M3, d["w13_scale"], adtype=orc.E4M3, a1=a1)
+    y = orc.expert_down(hq, offsets, d["w2"], orc.E4M3, d["w2_scale"], adtype=orc.E4M3, a2=a2)
+    xd = orc.e4m3_decode(xp) * a1
+    hd = orc.e4m3_decode(hq) * a2
+    for e in range(wl.E):
+        W1 = _decoded(d["w13"][e][:I], d["w13_scale"][e])
+        W3 = _decoded(d["w13"][e][I:], d["w13_scale"][e])
+        W2 = _decoded(d["w2"][e], d["w2_scale"][e])
+        for s in range(offsets[e], offsets[e + 1]):
+            g, u = W1 @ xd[s], W3 @ xd[s]
+            hr = g * expit(g) * u
+            assert np.allclose(h[s], hr, rtol=1e-12, atol=1e-14 * np.abs(hr).max())
+            yr = W2 @ hd[s]
+            assert np.allclose(y[s], yr, rtol=1e-12, atol=1e-14 * np.abs(yr).max())
