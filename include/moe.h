@@ -175,9 +175,14 @@ int moe_align_permute(const moe_shape_t *shape, const int32_t *ids, int32_t *cou
  *   device status (MOE_ERR_DEVICE_CHECK for an id outside 0..E-1).
  *   The first call on a device looks up the array's device address
  *   (cudaGetSymbolAddress) while that device is current; make that first call
- *   before any stream capture.  All calls share the one array, so calls that
+ *   before any stream capture.  The address is kept for the life of the
+ *   process: after cudaDeviceReset on a device, do not call this entry point
+ *   on that device again.  Devices with an index of 64 or more return
+ *   MOE_ERR_UNSUPPORTED.  All calls share the one array, so calls that
  *   overlap on the GPU (different streams, or different host threads using
- *   the same device) race and must be serialised by the caller.
+ *   the same device) race and must be serialised by the caller.  The status
+ *   word inside the array is cleared at the start of every call, so an error
+ *   reported by one call does not carry over to the next.
  */
 int moe_align_permute_noalloc(const moe_shape_t *shape, const int32_t *ids, int32_t *counts,
                               int32_t *offsets, int32_t *sorted_rows, int32_t *inv,
@@ -203,9 +208,11 @@ int moe_gather(const moe_shape_t *shape, const void *x, const int32_t *sorted_ro
  *   of each expert are W1 = gate, rows I..2I-1 are W3 = up), offsets as from
  *   step 2.  h [max_rows, I] out: bf16, or for adtype == MOE_E4M3 the E4M3
  *   codes of h / a2_scale (saturated).  Only rows of segments are written.
- *   fp32 accumulation in tensor memory; every weight byte of an expert is
- *   read once per call in the Swap-AB variant when the expert has at most
- *   256 rows.
+ *   fp32 accumulation in tensor memory.  In the Swap-AB variant an expert's
+ *   weight tile is streamed once per row tile of its segment: once when the
+ *   segment fits one tile (256 rows, or 64 rows for E4M3 weights with bf16
+ *   activations); the row tiles of one weight tile run side by side, so a
+ *   repeat read comes mostly from L2.
  *   E4M3 weights with bf16 activations (this call and step 5): the
  *   activation rows are first split, in the workspace, into two E4M3 planes
  *   with one power-of-two scale s per row, v = s * (hi + lo), and the GEMM

@@ -105,6 +105,9 @@ struct GemmPlan {
 };
 
 GemmPlan plan_gemm(const moe_shape_t &s);
+// Kernel launches issued by the last entry-point call on this host thread
+// (what moe_last_launch_count reports); every entry point resets it.
+int &launch_counter();
 bool ws_layout(const moe_shape_t &s, WsLayout &L);
 int validate_shape(const moe_shape_t *s, bool need_gemm);
 
@@ -117,10 +120,12 @@ cudaError_t launch_router(const moe_shape_t &s, const void *x, const void *wg, f
 // `chained`: launched by moe_fused_forward after its first kernel (PDL
 // launch; the control words and GEMM tile counters were zeroed at the start
 // of the call)
+// `ticket_zero`: the caller has already cleared ctrl->ticket on this stream
+// (skips the memset the two-kernel path otherwise issues)
 cudaError_t launch_align(const moe_shape_t &s, const int32_t *ids, int32_t *counts,
                          int32_t *offsets, int32_t *sorted_rows, int32_t *inv, int32_t *chunk_hist,
                          int32_t *chunk_base, Ctrl *ctrl, cudaStream_t st, int *launches,
-                         bool chained = false);
+                         bool chained = false, bool ticket_zero = false);
 cudaError_t launch_gather(const moe_shape_t &s, const void *x, const int32_t *sorted_rows,
                           const int32_t *offsets, float a1, void *xp, int64_t max_rows,
                           cudaStream_t st, bool chained = false);

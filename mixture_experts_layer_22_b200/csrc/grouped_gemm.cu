@@ -69,9 +69,8 @@ struct GemmParams {
 
 template <int kMode, bool kSwap, bool kFp8, int kBN, bool kHiLo = false, bool kPair = false>
 struct Cfg {
-    // K bytes per operand row and stage (128: the 128-byte swizzle; 64-byte
-    // rows with the 64-byte swizzle are supported by the loads and
-    // descriptors but measured slower for the normal order on B200).
+    // K bytes per operand row and stage: the 128-byte swizzle (64-byte rows
+    // with the 64-byte swizzle measured slower for the normal order on B200).
     static constexpr int kRowBytes = 128;
     static constexpr int kMmaPerStage = kRowBytes / 32;     // 32 bytes of K per MMA
     static constexpr int kStageA = 128 * kRowBytes;          // 128 rows
@@ -520,8 +519,8 @@ __global__ void __launch_bounds__(Cfg<kMode, kSwap, kFp8, kBN, kHiLo, kPair>::kT
                     const uint32_t sb = sa + C::kStageA;
 #pragma unroll
                     for (int s = 0; s < C::kMmaPerStage; ++s) {
-                        const uint64_t ad = C::kRowBytes == 128 ? sdesc_k_sw128(sa + s * 32) : sdesc_k_sw64(sa + s * 32);
-                        const uint64_t bd = C::kRowBytes == 128 ? sdesc_k_sw128(sb + s * 32) : sdesc_k_sw64(sb + s * 32);
+                        const uint64_t ad = sdesc_k_sw128(sa + s * 32);
+                        const uint64_t bd = sdesc_k_sw128(sb + s * 32);
                         const uint32_t accum = (kk > it.kb || s > 0) ? 1u : 0u;
                         if constexpr (kPair) {
                             if (kFp8) mma_e4m3_pair(d, ad, bd, idesc, accum);
@@ -856,8 +855,9 @@ static EncodeTiledFn get_encode_fn()
 // 2-D map over a row-major [rows, cols] matrix with 128-byte rows per box
 // and the 128-byte swizzle; box = box_rows x (128 bytes).
 static bool make_map(CUtensorMap *m, const void *base, bool u8, uint64_t rows, uint64_t cols,
-                     uint32_t box_rows, uint32_t row_bytes = 128)
+                     uint32_t box_rows)
 {
+    constexpr uint32_t row_bytes = 128;
     EncodeTiledFn fn = get_encode_fn();
     if (!fn) return false;
     const uint32_t esz = u8 ? 1 : 2;
@@ -867,7 +867,7 @@ static bool make_map(CUtensorMap *m, const void *base, bool u8, uint64_t rows, u
     cuuint32_t estr[2] = {1, 1};
     CUresult r = fn(m, u8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
                     const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                    row_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+                    CU_TENSOR_MAP_SWIZZLE_128B,
                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
@@ -939,8 +939,9 @@ static cudaError_t run_gemm(const moe_shape_t &s, const GemmArgs &a, cudaStream_
     const uint32_t wbox = kSwap ? (kMode == 0 ? 64 : 128) : (kMode == 0 || kPair ? 128 : 256);
     const uint32_t xbox = kSwap ? 16 : 128;     // Swap-AB loads token rows in 16-row boxes
     CUtensorMap tm_w, tm_x;
-    if (!make_map(&tm_w, a.wgt, u8w, Et * w_rows, K, wbox, Cf::kRowBytes) ||
-        !make_map(&tm_x, a.act, u8, Cf::kPlanes * a.max_rows, K, xbox, Cf::kRowBytes)) {
+    static_assert(Cf::kRowBytes == 128, "tensor maps use 128-byte rows with the 128-byte swizzle");
+    if (!make_map(&tm_w, a.wgt, u8w, Et * w_rows, K, wbox) ||
+        !make_map(&tm_x, a.act, u8, Cf::kPlanes * a.max_rows, K, xbox)) {
         *host_err = MOE_ERR_CUDA;
         return cudaSuccess;
     }

@@ -11,6 +11,8 @@ namespace moe {
 
 static thread_local int g_launches = 0;
 
+int &launch_counter() { return g_launches; }
+
 static size_t up256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
 int validate_shape(const moe_shape_t *s, bool need_gemm)
@@ -39,15 +41,21 @@ GemmPlan plan_gemm(const moe_shape_t &s)
     GemmPlan p;
     // One tcgen05.mma on one SM has a fixed 128-row M extent: when no expert
     // can receive 128 rows or more, weights go to M and tokens to N.
-    // E4M3 weights with bf16 activations are converted in the weight (M)
-    // slot, so that path is always Swap-AB.
+    // E4M3 weights with bf16 activations stack the hi and lo E4M3 planes of
+    // the activation rows in the MMA's N, so that path is always Swap-AB.
     p.swap = s.variant == MOE_VARIANT_SWAP_AB || (s.variant == MOE_VARIANT_AUTO && s.T <= 128) ||
              (s.wdtype == MOE_E4M3 && s.adtype == MOE_BF16);
     if (p.swap) {
         const int rows = (s.T + s.pad - 1) / s.pad * s.pad;   // worst case rows of one expert
         int bn = 16;
-        // the E4M3-weight path keeps converted weight slabs and split
-        // accumulators in tensor memory, which caps its token tile at 64 rows
+        // The hi/lo path holds two planes per token row, so a 64-row tile
+        // already stages and accumulates 128 columns.  The smem ring is sized
+        // per launch from the largest segment (the shared expert's T rows at
+        // T >= 64), and 64-row tiles keep 6 stages in flight where 128-row
+        // ones would keep 4 for the whole weight stream.  The price is that a
+        // segment of more than 64 rows takes two row tiles over the same
+        // weight tile; those are adjacent in the tile list, so they run at the
+        // same time and the second read comes mostly from L2.
         const int cap = (s.wdtype == MOE_E4M3 && s.adtype == MOE_BF16) ? 64 : 256;
         while (bn < rows && bn < cap) bn <<= 1;
         p.bn = bn;

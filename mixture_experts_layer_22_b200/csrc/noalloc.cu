@@ -33,11 +33,14 @@ constexpr int kMaxDevices = 64;
 static std::mutex g_setup_mutex;
 static void *g_scratch_addr[kMaxDevices];
 
-// Device address of g_align_scratch on the current device (looked up once).
+// Device address of g_align_scratch on the current device (looked up once per
+// device and kept for the life of the process: a cudaDeviceReset, which
+// unloads the library's module, makes the kept address stale).
 static int scratch_address(void **addr)
 {
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MOE_ERR_CUDA;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return MOE_ERR_CUDA;
+    if (dev >= kMaxDevices) return MOE_ERR_UNSUPPORTED;
     std::lock_guard<std::mutex> lock(g_setup_mutex);
     if (!g_scratch_addr[dev]) {
         void *p = nullptr;
@@ -56,6 +59,8 @@ extern "C" int moe_align_permute_noalloc(const moe_shape_t *shape, const int32_t
                                          int32_t *counts, int32_t *offsets, int32_t *sorted_rows,
                                          int32_t *inv, int32_t *status, moe_stream_t stream)
 {
+    int &launches = launch_counter();
+    launches = 0;
     int st = validate_shape(shape, false);
     if (st != MOE_OK) return st;
     if (!ids || !counts || !offsets || !sorted_rows || !inv) return MOE_ERR_INVALID_ARG;
@@ -70,11 +75,11 @@ extern "C" int moe_align_permute_noalloc(const moe_shape_t *shape, const int32_t
     int32_t *hist = reinterpret_cast<int32_t *>(b + kNoAllocCtrlBytes);
     int32_t *first = reinterpret_cast<int32_t *>(b + kNoAllocCtrlBytes + kNoAllocHistBytes);
     // the array keeps the previous call's contents: the status word and the
-    // blocks-finished ticket must start from zero
-    if (cudaMemsetAsync(ctrl, 0, sizeof(Ctrl), sm) != cudaSuccess) return MOE_ERR_CUDA;
-    int launches = 0;
-    if (launch_align(*shape, ids, counts, offsets, sorted_rows, inv, hist, first, ctrl, sm, &launches) !=
-        cudaSuccess)
+    // blocks-finished ticket (adjacent) must start from zero
+    static_assert(offsetof(Ctrl, ticket) == sizeof(int32_t), "status and ticket adjacent");
+    if (cudaMemsetAsync(ctrl, 0, 2 * sizeof(int32_t), sm) != cudaSuccess) return MOE_ERR_CUDA;
+    if (launch_align(*shape, ids, counts, offsets, sorted_rows, inv, hist, first, ctrl, sm, &launches, false,
+                     true) != cudaSuccess)
         return MOE_ERR_CUDA;
     if (status && cudaMemcpyAsync(status, &ctrl->status, sizeof(int32_t), cudaMemcpyDeviceToDevice, sm) !=
                       cudaSuccess)

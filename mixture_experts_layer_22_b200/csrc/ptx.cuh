@@ -201,13 +201,6 @@ __device__ __forceinline__ void prefetch_tmap(const CUtensorMap *map)
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
 
-// Make generic-proxy writes to shared memory visible to the async proxy
-// (tensor core operand reads).
-__device__ __forceinline__ void fence_proxy_async_smem()
-{
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-
 // ------------------------------------------------------------------ tcgen05
 __device__ __forceinline__ void tmem_alloc(uint32_t dst_smem, uint32_t ncols)
 {
@@ -267,19 +260,6 @@ __device__ __forceinline__ uint64_t sdesc_k_sw128(uint32_t saddr)
     d |= static_cast<uint64_t>(1024 >> 4) << 32;             // stride offset  [32,46)
     d |= static_cast<uint64_t>(1) << 46;                     // descriptor version (sm_100)
     d |= static_cast<uint64_t>(2) << 61;                     // 128-byte swizzle
-    return d;
-}
-
-// Same for a K-major tile stored with the 64-byte swizzle: rows of 64 bytes,
-// 8-row groups 512 bytes apart.
-__device__ __forceinline__ uint64_t sdesc_k_sw64(uint32_t saddr)
-{
-    uint64_t d = 0;
-    d |= static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4);   // start address  [0,14)
-    d |= static_cast<uint64_t>(1) << 16;                     // leading offset [16,30) (unused)
-    d |= static_cast<uint64_t>(512 >> 4) << 32;              // stride offset  [32,46)
-    d |= static_cast<uint64_t>(1) << 46;                     // descriptor version (sm_100)
-    d |= static_cast<uint64_t>(4) << 61;                     // 64-byte swizzle
     return d;
 }
 
@@ -368,47 +348,6 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16])
           "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
           "=r"(r[14]), "=r"(r[15])
         : "r"(taddr));
-}
-
-// 32 lanes x 32 columns store: thread i of the warp writes lane
-// (quarter*32 + i), columns [col, col+32).
-__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32])
-{
-    asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
-        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
-        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
-        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
-        "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]),
-        "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]),
-        "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
-        : "memory");
-}
-
-__device__ __forceinline__ void tmem_wait_st()
-{
-    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
-}
-
-// MMA with the A operand in tensor memory (128 lanes = 128 rows of A, K
-// packed two bf16 per 32-bit column) and B from shared memory.
-__device__ __forceinline__ void mma_bf16_tmem_a(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc,
-                                                uint32_t idesc, uint32_t accumulate)
-{
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
-
-// Two E4M3 codes (low byte = first) -> two fp16 values, exactly.
-__device__ __forceinline__ uint32_t cvt_e4m3x2_f16x2(uint16_t v)
-{
-    uint32_t r;
-    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(r) : "h"(v));
-    return r;
 }
 
 __device__ __forceinline__ void tmem_wait_ld()

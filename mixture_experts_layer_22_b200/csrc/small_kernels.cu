@@ -436,7 +436,8 @@ __global__ void __launch_bounds__(1024) align_single_kernel(const int32_t *__res
 
 cudaError_t launch_align(const moe_shape_t &s, const int32_t *ids, int32_t *counts,
                          int32_t *offsets, int32_t *sorted_rows, int32_t *inv, int32_t *chunk_hist,
-                         int32_t *chunk_base, Ctrl *ctrl, cudaStream_t st, int *launches, bool chained)
+                         int32_t *chunk_base, Ctrl *ctrl, cudaStream_t st, int *launches, bool chained,
+                         bool ticket_zero)
 {
     const int R = s.T * s.k, Et = s.E + s.n_shared;
     const int nb = (R + kAlignChunk - 1) / kAlignChunk;
@@ -453,7 +454,7 @@ cudaError_t launch_align(const moe_shape_t &s, const int32_t *ids, int32_t *coun
                              chained, ids, R, s.T, s.E, s.n_shared, s.pad, counts, offsets, sorted_rows, inv,
                              ctrl);
     }
-    if (!chained) {
+    if (!chained && !ticket_zero) {
         cudaError_t err = cudaMemsetAsync(&ctrl->ticket, 0, sizeof(int32_t), st);
         if (err != cudaSuccess) return err;
     }

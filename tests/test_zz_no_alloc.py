@@ -56,3 +56,35 @@ def test_noalloc_align_rejects_shapes_beyond_its_scratch():
     with pytest.raises(moe.MoeError) as e:
         moe.align_permute_noalloc(s, dummy, dummy, dummy, dummy, dummy)
     assert e.value.code == -2
+
+
+@pytest.mark.parametrize("T,E,k", [(64, 8, 2), (3000, 60, 4)])       # one-kernel and two-kernel paths
+def test_noalloc_align_reports_a_bad_id_then_starts_clean(T, E, k):
+    """An expert id outside 0..E-1 is reported through the optional status
+    output; the next call on the same shared array starts from a clear status
+    and matches moe_align_permute again.  The launch count is this call's."""
+    wl = syn.Workload("na", T=T, H=128, I=128, E=E, k=k)
+    s = moe.Shape.of(wl)
+    ids_np = _ids(T, E, k, 5)
+    bad = ids_np.copy()
+    bad[T // 2, 0] = E                                           # one id out of range
+    status = torch.full((1,), 99, dtype=torch.int32, device="cuda")
+    got = _buffers(s, T, k, E, 0)
+    moe.align_permute_noalloc(s, torch.from_numpy(bad).cuda(), *got, status)
+    torch.cuda.synchronize()
+    assert int(status[0]) == -5                                  # MOE_ERR_DEVICE_CHECK
+    assert moe.last_launch_count() == (1 if T * k <= 1024 else 2)
+    ids = torch.from_numpy(ids_np).cuda()
+    ref = _buffers(s, T, k, E, 0)
+    ws = moe.workspace(s)
+    moe.reset_device_status(ws)
+    moe.align_permute(s, ids, *ref, ws)
+    got = _buffers(s, T, k, E, 0)
+    moe.align_permute_noalloc(s, ids, *got, status)
+    torch.cuda.synchronize()
+    assert int(status[0]) == 0
+    total = int(ref[1][-1])
+    for g, r in zip(got[:2], ref[:2]):
+        assert torch.equal(g, r)
+    assert torch.equal(got[2][:total], ref[2][:total])
+    assert torch.equal(got[3], ref[3])
