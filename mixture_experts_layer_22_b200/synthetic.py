@@ -19,6 +19,9 @@ Workloads (the layer shapes the library is measured and checked on):
                        activations, static per-tensor scales
   dsv3_decode_fp8w     T=1/8/32/128 H=7168 I=2048 E=256 top-8 sigmoid x2.5
                        (renormalised) + 1 shared expert, E4M3 weights, bf16 acts
+  dsv3_decode_fp8      the same layer (same weights and tokens) with E4M3
+                       activations too: static per-tensor scales calibrated
+                       on the 128 seeded tokens
   qwen2_skewed_prefill T=8192 H=2048 I=1408 E=60 top-4 softmax, bf16, router
                        logits N(0,1) + Zipf(1.2) expert bias
 Distributions: x ~ N(0,1); router weight W_g ~ N(0, 0.02^2) in bf16 and
@@ -57,6 +60,8 @@ class Workload:
     logits: str = "router"          # "router" (x . W_g) or "zipf" (N(0,1) + bias)
     zipf_s: float = 1.2
     seed: int = 0
+    calib_T: int = 0                # E4M3 activations: a1 from the first calib_T tokens
+                                    # (0: from this batch's own T tokens)
 
     @property
     def E_tot(self) -> int:
@@ -73,6 +78,9 @@ WORKLOADS = {
                                     wdtype=E4M3, adtype=E4M3),
     "dsv3_decode_fp8w": Workload("dsv3_decode_fp8w", T=128, H=7168, I=2048, E=256, k=8,
                                  n_shared=1, gate=SIGMOID, routed_scale=2.5, wdtype=E4M3),
+    "dsv3_decode_fp8": Workload("dsv3_decode_fp8", T=128, H=7168, I=2048, E=256, k=8,
+                                n_shared=1, gate=SIGMOID, routed_scale=2.5, wdtype=E4M3, adtype=E4M3,
+                                calib_T=128),
     "qwen2_skewed_prefill": Workload("qwen2_skewed_prefill", T=8192, H=2048, I=1408, E=60, k=4,
                                      logits="zipf"),
 }
@@ -173,7 +181,10 @@ def make_inputs(wl: Workload, weights: bool = True) -> dict:
     if weights:
         d["w13"], d["w13_scale"] = expert_weights(wl, "w13")
         d["w2"], d["w2_scale"] = expert_weights(wl, "w2")
-    d["a1"] = activation_scale(x) if wl.adtype == E4M3 else 1.0
+    if wl.adtype == E4M3:
+        d["a1"] = activation_scale(x if not wl.calib_T else tokens(wl.with_T(wl.calib_T)))
+    else:
+        d["a1"] = 1.0
     return d
 
 
