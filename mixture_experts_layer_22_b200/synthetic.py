@@ -24,6 +24,9 @@ Workloads (the layer shapes the library is measured and checked on):
                        on the 128 seeded tokens
   qwen2_skewed_prefill T=8192 H=2048 I=1408 E=60 top-4 softmax, bf16, router
                        logits N(0,1) + Zipf(1.2) expert bias
+Attention side (the inverse-rotary + per-head E4M3 step): rope_mixtral (32
+heads x 128, neox pairs, base 1e6) and rope_dsv3 (128 heads x 64, interleaved
+pairs, base 1e4), T tokens at uniform random positions.
 Distributions: x ~ N(0,1); router weight W_g ~ N(0, 0.02^2) in bf16 and
 logits = fp32(x . W_g^T) computed in double; expert weights ~ N(0, 1/fan_in)
 (standard deviation 1/sqrt(fan_in), fan_in = H for W1/W3 and I for W2).
@@ -186,6 +189,53 @@ def make_inputs(wl: Workload, weights: bool = True) -> dict:
     else:
         d["a1"] = 1.0
     return d
+
+
+# ---------------------------------------------------------------- attention side
+@dataclasses.dataclass(frozen=True)
+class RopeWorkload:
+    """Inputs of the inverse-rotary + per-head E4M3 step: T tokens of n_heads
+    vectors of head_dim, the first rot_dim of which carry the rotation."""
+    name: str
+    T: int
+    n_heads: int
+    head_dim: int
+    rot_dim: int
+    interleaved: bool = False
+    base: float = 1.0e6
+    max_pos: int = 32768
+    seed: int = 0
+
+    def with_T(self, T: int) -> "RopeWorkload":
+        return dataclasses.replace(self, T=T)
+
+
+ROPE_WORKLOADS = {
+    # Mixtral-shaped attention (32 heads of 128, rotary base 1e6, neox pairs)
+    "rope_mixtral": RopeWorkload("rope_mixtral", T=8192, n_heads=32, head_dim=128, rot_dim=128),
+    # DeepSeek-V3-shaped rotary part (128 heads of 64, interleaved pairs)
+    "rope_dsv3": RopeWorkload("rope_dsv3", T=8192, n_heads=128, head_dim=64, rot_dim=64, interleaved=True,
+                              base=1.0e4, max_pos=163840),
+}
+
+
+def rope_table(rw: RopeWorkload) -> np.ndarray:
+    """The model's rotary table cos_sin [max_pos, rot_dim] fp32: row p holds
+    cos(p w_i) for i < rot_dim/2 then sin(p w_i), w_i = base^(-2i/rot_dim),
+    evaluated in double and rounded once (a constant of the model, built at
+    start-up like its weights)."""
+    half = rw.rot_dim // 2
+    w = rw.base ** (-2.0 * np.arange(half, dtype=np.float64) / rw.rot_dim)
+    ang = np.arange(rw.max_pos, dtype=np.float64)[:, None] * w[None, :]
+    return np.concatenate([np.cos(ang), np.sin(ang)], axis=1).astype(np.float32)
+
+
+def rope_inputs(rw: RopeWorkload) -> dict:
+    """x [T, n_heads, head_dim] bf16 bits ~ N(0, 1), positions [T] int32
+    uniform in [0, max_pos), and the rotary table."""
+    x = to_bf16_bits(_normal(rw.seed, "rope_x", 0, (rw.T, rw.n_heads, rw.head_dim), 1.0))
+    pos = _rng(rw.seed, "rope_pos").integers(0, rw.max_pos, size=rw.T, dtype=np.int32)
+    return {"x": x, "positions": pos, "cos_sin": rope_table(rw)}
 
 
 def random_rows(seed: int, name: str, rows: int, cols: int, dtype: int, std: float = 1.0):

@@ -30,10 +30,11 @@ _lib = None
 
 
 def build(force: bool = False) -> str:
-    """Compile the oracle with gcc (-O2, OpenMP, no fast-math)."""
+    """Compile the oracle with gcc (-O2, OpenMP, no fast-math, no contraction of
+    a * b + c into a fused multiply-add)."""
     if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
         tmp = _LIB + f".tmp{os.getpid()}"
-        subprocess.check_call(["gcc", "-O2", "-fopenmp", "-fno-fast-math", "-shared", "-fPIC",
+        subprocess.check_call(["gcc", "-O2", "-fopenmp", "-fno-fast-math", "-ffp-contract=off", "-shared", "-fPIC",
                                "-o", tmp, _SRC, "-lm"])
         os.replace(tmp, _LIB)
     return _LIB
@@ -73,6 +74,8 @@ def _load():
                                         d, d, P, l, P]
             lib.orc_hidden_amax.restype = d
             lib.orc_hidden_amax.argtypes = [i, i, i, i, i, i, i, d, i, i, P, P, P, P, d, P, l]
+            lib.orc_inv_rope_quant.restype = None
+            lib.orc_inv_rope_quant.argtypes = [i, i, i, i, i, P, P, P, i, P, P]
             lib.orc_num_threads.restype = i
             lib.orc_num_threads.argtypes = []
             _lib = lib
@@ -252,3 +255,22 @@ def hidden_amax(x_bits, logits, w13, *, E: int, k: int, n_shared: int = 0, gate:
     return _load().orc_hidden_amax(H, I, E, k, n_shared, gate, int(renorm), routed_scale, wdtype,
                                    adtype, _p(x_bits), _p(lg), _p(w13), _p(s13), a1, _p(toks),
                                    toks.size)
+
+
+# ---------------------------------------------------------------- attention side
+def inv_rope_quant(x_bits, positions, cos_sin, rot_dim: int, interleaved: bool = False):
+    """Inverse rotary embedding then per-head E4M3 quantisation.
+    x_bits [T, n_heads, head_dim] bf16 bits, positions [T] int32, cos_sin
+    [max_pos, rot_dim] fp32; returns (codes [T, n_heads, head_dim] uint8,
+    scales [T, n_heads] fp32)."""
+    xb = _c(x_bits, np.uint16)
+    T, nh, hd = xb.shape
+    pos = _c(positions, np.int32)
+    cs = _c(cos_sin, np.float32)
+    if cs.shape[1] != rot_dim or rot_dim % 2 or rot_dim > hd or pos.shape != (T,):
+        raise ValueError("cos_sin [max_pos, rot_dim], even rot_dim <= head_dim, positions [T] expected")
+    q = np.empty((T, nh, hd), dtype=np.uint8)
+    sc = np.empty((T, nh), dtype=np.float32)
+    _load().orc_inv_rope_quant(T, nh, hd, rot_dim, int(interleaved), _p(xb), _p(pos), _p(cs), cs.shape[0],
+                               _p(q), _p(sc))
+    return q, sc

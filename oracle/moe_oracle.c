@@ -500,6 +500,80 @@ double orc_hidden_amax(int H, int I, int E, int k, int n_shared, int gate,
     return amax;
 }
 
+/* ------------------------------------------------------------------------ */
+/* inverse rotary embedding + per-head E4M3 quantisation (attention side)    */
+/* ------------------------------------------------------------------------ */
+
+/* The Russian summary, section "Убрать лишние JIT-перекомпиляции Triton",
+ * names a kernel that fuses rotary position embedding with FP8 quantisation
+ * per head and must take the token count as a run-time value.  The pages say
+ * nothing more, so the plain reading is:
+ *   - x [T, n_heads, head_dim] bf16 holds vectors that carry the rotary
+ *     rotation of their token's position p (forward RoPE: each pair (a, b)
+ *     became (a c - b s, b c + a s) with c = cos(p w_i), s = sin(p w_i));
+ *   - the inverse rotation undoes it: a = a' c + b' s, b = b' c - a' s;
+ *   - pairs are (i, i + rot_dim/2) (the "neox" layout) or (2i, 2i+1)
+ *     (interleaved), over the first rot_dim elements; the rest pass through;
+ *   - c and s come from a table cos_sin [max_pos, rot_dim]: row p holds
+ *     cos(p w_i) for i < rot_dim/2, then sin(p w_i);
+ *   - each (token, head) vector r is then quantised to E4M3 with its own
+ *     scale = amax(|r|)/448 (1 when r is all zero): code = e4m3(r / scale).
+ * Every code is an integer decided by floating point, so the arithmetic is
+ * fixed in fp32 as the kernel does it: each product rounded, then the sum or
+ * difference rounded (no fused multiply-add), the scale and the quotient by
+ * IEEE fp32 division, then round-to-nearest-even with saturation to +-448.
+ * A position outside [0, max_pos) gives zero codes and scale 0. */
+void orc_inv_rope_quant(int T, int n_heads, int head_dim, int rot_dim, int interleaved,
+                        const uint16_t *x, const int32_t *pos, const float *cos_sin, int max_pos,
+                        uint8_t *q, float *scale)
+{
+    const int half = rot_dim / 2;
+#pragma omp parallel for schedule(static)
+    for (long th = 0; th < (long)T * n_heads; ++th) {
+        const long t = th / n_heads;
+        const uint16_t *xh = x + th * head_dim;
+        uint8_t *qh = q + th * head_dim;
+        const int p = pos[t];
+        if (p < 0 || p >= max_pos) {
+            for (int j = 0; j < head_dim; ++j) qh[j] = 0;
+            scale[th] = 0.0f;
+            continue;
+        }
+        const float *cs = cos_sin + (long)p * rot_dim;
+        float *r = malloc(sizeof(float) * (size_t)head_dim);
+        float amax = 0.0f;
+        for (int j = 0; j < head_dim; ++j) {
+            const float y = (float)orc_bf16_decode(xh[j]);
+            float v = y;
+            if (j < rot_dim) {
+                int i, partner, first;
+                if (interleaved) {
+                    i = j / 2;
+                    first = (j % 2) == 0;
+                    partner = first ? j + 1 : j - 1;
+                } else {
+                    first = j < half;
+                    i = first ? j : j - half;
+                    partner = first ? j + half : j - half;
+                }
+                const float yp = (float)orc_bf16_decode(xh[partner]);
+                const float a = y * cs[i];
+                const float b = yp * cs[half + i];
+                v = first ? a + b : a - b;
+            }
+            r[j] = v;
+            if (fabsf(v) > amax) amax = fabsf(v);
+        }
+        const float sc = amax > 0.0f ? amax / 448.0f : 1.0f;
+        scale[th] = sc;
+        for (int j = 0; j < head_dim; ++j) {
+            const float quot = r[j] / sc;
+            qh[j] = orc_e4m3_encode((double)quot);
+        }
+        free(r);
+    }
+}
+
 int orc_num_threads(void)
 {
 #ifdef _OPENMP

@@ -1,6 +1,7 @@
 """Pins for the CPU oracle: each test checks the oracle against something other
 than itself -- a format definition, a library routine the case reduces to, a
 closed form, an invariant, or brute force on tiny inputs.  CPU only."""
+import dataclasses
 import itertools
 
 import numpy as np
@@ -489,3 +490,110 @@ def test_fp8_expert_gemm_references_row_by_row():
             assert np.allclose(h[s], hr, rtol=1e-12, atol=1e-14 * np.abs(hr).max())
             yr = W2 @ hd[s]
             assert np.allclose(y[s], yr, rtol=1e-12, atol=1e-14 * np.abs(yr).max())
+
+
+# ------------------------------------------------------------------ inverse rotary + per-head E4M3
+# The Russian summary (section "Убрать лишние JIT-перекомпиляции Triton")
+# names a fused rotary-embedding + per-head FP8 quantisation kernel.  These
+# pins tie the oracle's reading (inverse rotation, neox or interleaved pairs,
+# scale = amax/448 per head) to a right-angle rotation, the identity at
+# position 0, scipy's rotation matrices, and a layout permutation.
+def _rope_case(T=6, nh=3, hd=16, rot=16, seed=31):
+    rw = syn.RopeWorkload("pin", T=T, n_heads=nh, head_dim=hd, rot_dim=rot, max_pos=64, base=1e4, seed=seed)
+    return rw, syn.rope_inputs(rw)
+
+
+def _head_scale(v):
+    amax = np.float32(np.max(np.abs(v)))
+    return np.float32(amax / np.float32(448.0)) if amax > 0 else np.float32(1.0)
+
+
+def test_inv_rope_position_zero_is_plain_per_head_quantisation():
+    rw, d = _rope_case()
+    pos = np.zeros(rw.T, np.int32)
+    q, sc = orc.inv_rope_quant(d["x"], pos, d["cos_sin"], rw.rot_dim)
+    xf = syn.bf16_bits_to_f32(d["x"])
+    for t in range(rw.T):
+        for h in range(rw.n_heads):
+            s = _head_scale(xf[t, h])
+            assert sc[t, h] == s
+            assert np.array_equal(q[t, h], orc.quant_e4m3_f32(xf[t, h], float(s)))
+
+
+@pytest.mark.parametrize("interleaved", [False, True])
+def test_inv_rope_right_angle_swaps_and_negates(interleaved):
+    """A table row with cos = 0, sin = 1 exactly (a quarter turn): the inverse
+    rotation maps each pair (a', b') to (b', -a')."""
+    rw, d = _rope_case()
+    cs = np.zeros((2, rw.rot_dim), np.float32)
+    cs[1, rw.rot_dim // 2:] = 1.0
+    pos = np.ones(rw.T, np.int32)
+    q, sc = orc.inv_rope_quant(d["x"], pos, cs, rw.rot_dim, interleaved)
+    xf = syn.bf16_bits_to_f32(d["x"])
+    half = rw.rot_dim // 2
+    r = np.empty_like(xf)
+    for i in range(half):
+        a, b = (2 * i, 2 * i + 1) if interleaved else (i, i + half)
+        r[..., a] = xf[..., b]
+        r[..., b] = -xf[..., a]
+    for t in range(rw.T):
+        for h in range(rw.n_heads):
+            s = _head_scale(r[t, h])
+            assert sc[t, h] == s
+            assert np.array_equal(q[t, h], orc.quant_e4m3_f32(r[t, h], float(s)))
+
+
+def test_inv_rope_matches_scipy_rotation_by_minus_theta():
+    """General angles: each pair rotated by -theta (theta from the table's
+    cos/sin) with scipy's rotation matrices, in double; the oracle's codes
+    decode to it within half an E4M3 step (plus fp32 rounding)."""
+    from scipy.spatial.transform import Rotation
+    rw, d = _rope_case(T=12, nh=2, hd=32, rot=32, seed=33)
+    q, sc = orc.inv_rope_quant(d["x"], d["positions"], d["cos_sin"], rw.rot_dim)
+    xf = syn.bf16_bits_to_f32(d["x"]).astype(np.float64)
+    half = rw.rot_dim // 2
+    for t in range(rw.T):
+        row = d["cos_sin"][d["positions"][t]].astype(np.float64)
+        theta = np.arctan2(row[half:], row[:half])
+        for h in range(rw.n_heads):
+            ref = np.empty(rw.head_dim)
+            for i in range(half):
+                v = np.array([xf[t, h, i], xf[t, h, i + half], 0.0])
+                a, b, _ = Rotation.from_euler("z", -theta[i]).apply(v)
+                ref[i], ref[i + half] = a, b
+            got = orc.e4m3_decode(q[t, h]) * float(sc[t, h])
+            step = np.exp2(np.floor(np.log2(np.maximum(np.abs(ref), 1e-30) / sc[t, h]))) * 2.0 ** -3
+            tol = 0.5 * np.maximum(step, 2.0 ** -9) * sc[t, h] + 1e-5 * np.abs(ref).max()
+            assert np.all(np.abs(got - ref) <= tol)
+            assert np.abs(got).max() == pytest.approx(448.0 * float(sc[t, h]), rel=0, abs=0)
+
+
+def test_inv_rope_neox_and_interleaved_layouts_are_a_permutation_apart():
+    rw, d = _rope_case(T=8, nh=4, hd=32, rot=24, seed=35)
+    half = rw.rot_dim // 2
+    perm = np.arange(rw.head_dim)                 # interleaved slot -> neox slot
+    perm[0:rw.rot_dim:2] = np.arange(half)
+    perm[1:rw.rot_dim:2] = np.arange(half) + half
+    q_n, s_n = orc.inv_rope_quant(d["x"], d["positions"], d["cos_sin"][:, :rw.rot_dim], rw.rot_dim, False)
+    q_i, s_i = orc.inv_rope_quant(d["x"][..., perm], d["positions"], d["cos_sin"][:, :rw.rot_dim], rw.rot_dim, True)
+    assert np.array_equal(s_n, s_i)
+    assert np.array_equal(q_n[..., perm], q_i)
+
+
+def test_inv_rope_partial_rotary_passes_the_rest_through():
+    rw, d = _rope_case(T=5, nh=2, hd=32, rot=16, seed=37)
+    cs = syn.rope_table(dataclasses.replace(rw, rot_dim=16))
+    q, sc = orc.inv_rope_quant(d["x"], d["positions"], cs, 16)
+    xf = syn.bf16_bits_to_f32(d["x"])
+    for t in range(rw.T):
+        for h in range(rw.n_heads):
+            assert np.array_equal(q[t, h, 16:], orc.quant_e4m3_f32(xf[t, h, 16:], float(sc[t, h])))
+
+
+def test_inv_rope_position_out_of_range_gives_zero_codes_and_scale():
+    rw, d = _rope_case()
+    pos = d["positions"].copy()
+    pos[2], pos[4] = -1, 64
+    q, sc = orc.inv_rope_quant(d["x"], pos, d["cos_sin"], rw.rot_dim)
+    assert np.all(q[[2, 4]] == 0) and np.all(sc[[2, 4]] == 0)
+    assert np.all(sc[[0, 1, 3, 5]] > 0)
