@@ -382,8 +382,11 @@ void orc_combine(int T, int H, int k, int E, int n_shared, const int32_t *offset
 /* ------------------------------------------------------------------------ */
 
 /* One expert's SwiGLU MLP on one token vector x (already in double).
- * adtype == E4M3: the token vector was quantised with a1 by the caller, and
- * the hidden vector h is quantised here: h_q = e4m3(h / a2) * a2. */
+ * The hidden vector h is an activation of the layer and is stored in the
+ * layer's activation dtype before the down projection reads it, as the token
+ * vector is: adtype == BF16 rounds h to bf16 (nearest even); adtype == E4M3
+ * (the token vector was quantised with a1 by the caller) quantises it,
+ * h_q = e4m3(h / a2) * a2.  Everything else is double. */
 static void expert_mlp(int H, int I, int e, const double *x,
                        const void *w13, const void *w2, int wdtype,
                        const float *w13_scale, const float *w2_scale,
@@ -400,6 +403,7 @@ static void expert_mlp(int H, int I, int e, const double *x,
         }
         double hv = silu(g * s1) * (u * s1);
         if (adtype == ORC_E4M3) hv = orc_e4m3_decode(orc_e4m3_encode(hv / a2)) * a2;
+        else hv = orc_bf16_decode(orc_bf16_encode(hv));
         hbuf[i] = hv;
     }
     for (int o = 0; o < H; ++o) {

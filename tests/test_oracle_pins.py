@@ -192,10 +192,18 @@ def test_align_empty_experts_and_one_hot_expert():
 
 
 # ------------------------------------------------------------------ expert math
-def _dense_swiglu(xd, W1, W3, W2):
+def _bf16_round(v):
+    """Round to bf16, nearest even (the library's cast), back to double."""
+    return torch.from_numpy(np.asarray(v, dtype=np.float64)).to(torch.bfloat16).double().numpy()
+
+
+def _dense_swiglu(xd, W1, W3, W2, round_h=True):
+    """The textbook dense SwiGLU MLP; the hidden vector, an activation of a
+    bf16 layer, is stored in bf16 (round_h) before the down projection."""
     g = xd @ W1.T
     u = xd @ W3.T
-    return (g * expit(g) * u) @ W2.T
+    h = g * expit(g) * u
+    return (_bf16_round(h) if round_h else h) @ W2.T
 
 
 def test_single_expert_top1_is_dense_swiglu_mlp():
@@ -235,7 +243,7 @@ def test_scalar_layer_closed_form():
     xs = np.array([-3.0, -0.5, 0.0, 0.75, 2.0, 6.0])
     x = bits(xs).reshape(-1, 1)
     out = orc.forward(x, np.zeros((6, 1), np.float32), w13, w2, E=1, k=1)[:, 0]
-    ref = c * (a * xs) * expit(a * xs) * (b * xs)
+    ref = c * _bf16_round((a * xs) * expit(a * xs) * (b * xs))
     assert np.allclose(out, ref, rtol=1e-14, atol=1e-15)
 
 
@@ -247,8 +255,8 @@ def test_row_wise_pieces_compose_to_dense_definition():
     counts, offsets, rows, inv = orc.align(ids, 5, 1, 8)
     xp = orc.gather(d["x"], rows, 2, 20, 1)
     h = orc.expert_swiglu(xp, offsets, d["w13"], orc.BF16)
-    # compose in double: h itself (not rounded to bf16) goes through the down step
-    y = _down_double(h, offsets, d["w2"])
+    # h is stored as bf16 between the two steps, as in the layer
+    y = orc.expert_down(orc.bf16_encode(h), offsets, d["w2"], orc.BF16)
     out = orc.combine(y, w, inv, offsets, 5, 1)
     ref = orc.forward(d["x"], d["logits"], d["w13"], d["w2"], E=5, k=2, n_shared=1,
                       gate=orc.SIGMOID, routed_scale=2.5)
