@@ -8,7 +8,8 @@ moe_fused_forward per step with inputs resident in HBM.  At N=1 the same JSON
 line also carries `per_workload`, the same measurements for every other
 configuration (tiny layer; Mixtral decode T=1/8/64; Mixtral E4M3 prefill
 T=4096; DeepSeek-V3 decode T=1/8/32, with E4M3 weights and with E4M3
-activations too; Qwen2-MoE skewed prefill T=8192).  Prints one JSON line.
+activations too; Qwen2-MoE skewed prefill T=8192) and for the attention-side
+inverse-rotary + per-head E4M3 step.  Prints one JSON line.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                   [--workload NAME] [--T T] [--no-sweep]
@@ -300,10 +301,26 @@ class DeviceLayer:
         torch.cuda.synchronize(self.dev)
 
     def step(self, graph=True):
-        if graph:
-            self.graph.replay()
-        else:
-            self.call()
+        # a graph replays on torch's current stream: make that the layer's stream
+        with self.torch.cuda.stream(self.stream):
+            if graph:
+                self.graph.replay()
+            else:
+                self.call()
+
+    def check_graph_matches_direct(self):
+        """The replayed graph does the layer's work: its output equals a direct
+        call's, bit for bit."""
+        torch = self.torch
+        self.out.fill_(0)
+        self.step(True)
+        torch.cuda.synchronize(self.dev)
+        g = self.out.clone()
+        self.out.fill_(0)
+        self.call()
+        torch.cuda.synchronize(self.dev)
+        if not torch.equal(g.view(torch.int16), self.out.view(torch.int16)):
+            raise SystemExit(f"{self.wl.name} T={self.wl.T}: graph replay output differs from a direct call")
 
     def routing_facts(self):
         """Distinct active experts (routed with >= 1 row, plus shared) and
@@ -428,10 +445,11 @@ def time_e2e(L, steps, warmup, graph):
         ev_in[b].record(s_in)
         L.stream.wait_event(ev_in[b])
         L.stream.wait_event(ev_out[b])        # step i-2's D2H is done reading dout[b]
-        if graphs[b] is not None:
-            graphs[b].replay()
-        else:
-            L.call(dx[b], dl[b], dout[b])
+        with torch.cuda.stream(L.stream):
+            if graphs[b] is not None:
+                graphs[b].replay()
+            else:
+                L.call(dx[b], dl[b], dout[b])
         ev_layer[b].record(L.stream)
         s_out.wait_event(ev_layer[b])
         with torch.cuda.stream(s_out):
@@ -472,6 +490,7 @@ def measure_workload(wl, d, dev, args, weights=None, full=False, flush=None):
     st = L.moe.device_status(L.ws, L.stream)
     if st != 0:
         raise SystemExit(f"{wl.name} T={wl.T}: device status after warm-up: {L.moe.status_string(st)}")
+    L.check_graph_matches_direct()
     # flush L2 between steps when the weights of one step would stay in it
     wbytes = active * weight_bytes_per_expert(wl)
     use_flush = flush if (flush is not None and wbytes < 4 * L2_BYTES) else None
@@ -551,6 +570,7 @@ def ours_main(args, wl):
     st = L.moe.device_status(L.ws, L.stream)
     if st != 0:
         raise SystemExit(f"device status after warm-up: {L.moe.status_string(st)}")
+    L.check_graph_matches_direct()
 
     # clocks: sampled through a soak of about half a second of steps and the
     # timed region right after it
@@ -636,6 +656,49 @@ def ours_main(args, wl):
     return 0
 
 
+ROPE_SWEEP = [("rope_mixtral", 8192), ("rope_mixtral", 64), ("rope_dsv3", 8192)]
+
+
+def measure_rope(rw, dev, args, flush):
+    """The attention-side step (inverse rotary + per-head E4M3, one launch):
+    tokens/s and HBM GB/s of its algorithmic bytes (x in, codes and scales
+    out, positions and the table rows it reads), each step timed alone with L2
+    rewritten in between (its data fits in L2)."""
+    import torch
+    import mixture_experts_layer_22_b200 as moe
+    d = syn.rope_inputs(rw)
+    s = moe.RopeShape.of(rw)
+    x = torch.from_numpy(d["x"].view(np.int16)).to(dev).view(torch.bfloat16)
+    pos = torch.from_numpy(d["positions"]).to(dev)
+    cs = torch.from_numpy(d["cos_sin"]).to(dev)
+    q = torch.empty((rw.T, rw.n_heads, rw.head_dim), dtype=torch.uint8, device=dev)
+    sc = torch.empty((rw.T, rw.n_heads), dtype=torch.float32, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    st = torch.cuda.Stream(dev)
+    for _ in range(args.warmup):
+        moe.inv_rope_quant(s, x, pos, cs, q, sc, status, st)
+    torch.cuda.synchronize(dev)
+    if int(status.item()) != 0:
+        raise SystemExit(f"{rw.name}: device status {int(status.item())}")
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    for a, b in ev:
+        with torch.cuda.stream(st):
+            flush.add_(1)
+        a.record(st)
+        moe.inv_rope_quant(s, x, pos, cs, q, sc, status, st)
+        b.record(st)
+    torch.cuda.synchronize(dev)
+    ms = sum(a.elapsed_time(b) for a, b in ev) / args.steps
+    heads = rw.T * rw.n_heads
+    nbytes = heads * rw.head_dim * 3 + heads * 4 + rw.T * 4 + rw.T * rw.rot_dim * 4
+    hbm_peak = measured_peaks()[0]
+    return {"T": rw.T, "n_heads": rw.n_heads, "head_dim": rw.head_dim, "rot_dim": rw.rot_dim,
+            "interleaved": rw.interleaved, "ms_per_step": ms, "tokens_per_s": rw.T / (ms * 1e-3),
+            "roofline": {"bound": "hbm", "achieved": nbytes / (ms * 1e-3) / 1e9, "peak": hbm_peak, "unit": "GB/s",
+                         "frac": nbytes / (ms * 1e-3) / 1e9 / hbm_peak, "algorithmic_bytes": nbytes},
+            "l2": "flushed between timed steps", "launches_per_step": 1}
+
+
 def sweep(args, dev, d_head, weights_head, wl_head):
     """Every configuration besides the headline, measured the same way."""
     import torch
@@ -664,6 +727,11 @@ def sweep(args, dev, d_head, weights_head, wl_head):
         cache["weights"] = L.weights
         out[f"{wl.name} T={wl.T}"] = res
         del L
+    cache["weights"] = None
+    torch.cuda.empty_cache()
+    for name, T in ROPE_SWEEP:
+        rw = syn.ROPE_WORKLOADS[name].with_T(T)
+        out[f"{rw.name} T={rw.T}"] = measure_rope(rw, dev, args, flush)
     out["_clocks"] = clocks.stop()
     return out
 

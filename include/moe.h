@@ -268,6 +268,47 @@ int moe_fused_forward_router(const moe_shape_t *shape, const void *x, const void
                              moe_stream_t stream);
 
 /*
+ * Attention-side step: inverse rotary embedding fused with per-head E4M3
+ * quantisation ("_fused_inv_rope_fp8_quant_per_head" in the Russian summary,
+ * section "Убрать лишние JIT-перекомпиляции Triton": rotary embedding and FP8
+ * quantisation in one kernel, whose recompilation for every new num_tokens
+ * cost 9% of time-to-first-token until the token count was made a run-time
+ * value).  num_tokens is a run-time value here; nothing is built per count.
+ *   num_tokens  tokens (>= 0; 0 is a no-op)
+ *   n_heads     heads per token (>= 1)
+ *   head_dim    64, 128 or 256
+ *   rot_dim     rotated elements per head, at most head_dim: even for
+ *               interleaved pairs, a multiple of 16 for neox pairs
+ *               (MOE_ERR_UNSUPPORTED otherwise); the rest pass through
+ *               unrotated
+ *   max_pos     rows of the rotary table
+ *   interleaved 0: pairs (i, i + rot_dim/2) ("neox"); 1: pairs (2i, 2i+1)
+ */
+typedef struct {
+    int32_t num_tokens, n_heads, head_dim, rot_dim, max_pos, interleaved;
+} moe_rope_shape_t;
+
+/*
+ *   x [num_tokens, n_heads, head_dim] bf16 (16-byte aligned), positions
+ *   [num_tokens] int32, cos_sin [max_pos, rot_dim] fp32 (row p: cos(p w_i)
+ *   for i < rot_dim/2, then sin(p w_i)) in; q [num_tokens, n_heads, head_dim]
+ *   E4M3 codes (8-byte aligned) and scales [num_tokens, n_heads] fp32 out.
+ *   Each pair (a', b') of a head is rotated back by its token's angle,
+ *   a = a' c + b' s, b = b' c - a' s; then scale = amax(|r|)/448 per (token,
+ *   head) (1 if all zero) and q = E4M3(r / scale), round to nearest even,
+ *   saturated.  fp32 arithmetic, each product and sum rounded on its own, IEEE
+ *   division: the codes are reproducible bit for bit.
+ *   status: optional device int32 (may be NULL); a position outside
+ *   [0, max_pos) sets it to MOE_ERR_DEVICE_CHECK (if it was 0) and gives that
+ *   token zero codes and scale 0.  Otherwise it is left unchanged.
+ * Errors: MOE_ERR_INVALID_ARG (bad sizes, NULL or misaligned pointers),
+ * MOE_ERR_UNSUPPORTED (other head_dim).  Asynchronous on `stream`.
+ */
+int moe_inv_rope_quant_per_head(const moe_rope_shape_t *shape, const void *x, const int32_t *positions,
+                                const float *cos_sin, uint8_t *q, float *scales, int32_t *status,
+                                moe_stream_t stream);
+
+/*
  * Self-test of the failure path (no counterpart on the pages): launches one
  * block whose two bounded pipeline waits run out, because nothing arrives on
  * their barriers.  The first gives up after the library's wait limit (2 s),

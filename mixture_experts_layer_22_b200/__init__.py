@@ -30,7 +30,7 @@ EXPORTS = ["moe_max_rows", "moe_workspace_size", "moe_route_topk", "moe_align_pe
            "moe_grouped_gemm_swiglu", "moe_grouped_gemm_down", "moe_combine", "moe_fused_forward",
            "moe_get_device_status", "moe_reset_device_status", "moe_status_string",
            "moe_last_launch_count", "moe_align_permute_noalloc", "moe_router_topk",
-           "moe_fused_forward_router", "moe_selftest_wait_timeout"]
+           "moe_fused_forward_router", "moe_selftest_wait_timeout", "moe_inv_rope_quant_per_head"]
 
 
 class MoeError(RuntimeError):
@@ -51,6 +51,17 @@ class Shape(C.Structure):
         return cls(T=wl.T if T is None else T, H=wl.H, I=wl.I, E=wl.E, k=wl.k, n_shared=wl.n_shared,
                    gate=wl.gate, renorm=int(wl.renorm), routed_scale=wl.routed_scale,
                    wdtype=wl.wdtype, adtype=wl.adtype, pad=pad, variant=variant)
+
+
+class RopeShape(C.Structure):
+    """Mirror of moe_rope_shape_t."""
+    _fields_ = [("num_tokens", C.c_int32), ("n_heads", C.c_int32), ("head_dim", C.c_int32),
+                ("rot_dim", C.c_int32), ("max_pos", C.c_int32), ("interleaved", C.c_int32)]
+
+    @classmethod
+    def of(cls, rw, T: int | None = None) -> "RopeShape":
+        return cls(num_tokens=rw.T if T is None else T, n_heads=rw.n_heads, head_dim=rw.head_dim,
+                   rot_dim=rw.rot_dim, max_pos=rw.max_pos, interleaved=int(rw.interleaved))
 
 
 _lib = None
@@ -83,6 +94,7 @@ def lib() -> C.CDLL:
             "moe_router_topk": [S, P, P, P, P, P, P, C.c_size_t, P],
             "moe_fused_forward_router": [S, P, P, P, P, P, P, C.c_float, C.c_float, P, P, C.c_size_t, P],
             "moe_selftest_wait_timeout": [P, P, P],
+            "moe_inv_rope_quant_per_head": [C.POINTER(RopeShape), P, P, P, P, P, P, P],
         }
         for name, args in sig.items():
             fn = getattr(L, name)
@@ -200,6 +212,13 @@ def fused_forward_router(shape, x, wg, w13, w13_scale, w2, w2_scale, a1, a2, out
     _check(lib().moe_fused_forward_router(C.byref(shape), _ptr(x), _ptr(wg), _ptr(w13), _ptr(w13_scale),
                                           _ptr(w2), _ptr(w2_scale), a1, a2, _ptr(out), _ptr(ws), ws.numel(),
                                           _stream(stream)), "moe_fused_forward_router")
+
+
+def inv_rope_quant(shape, x, positions, cos_sin, q, scales, status=None, stream=None):
+    """Inverse rotary embedding + per-head E4M3 quantisation (one launch)."""
+    _check(lib().moe_inv_rope_quant_per_head(C.byref(shape), _ptr(x), _ptr(positions), _ptr(cos_sin), _ptr(q),
+                                             _ptr(scales), _ptr(status), _stream(stream)),
+           "moe_inv_rope_quant_per_head")
 
 
 def selftest_wait_timeout(ws, gave_up, stream=None):

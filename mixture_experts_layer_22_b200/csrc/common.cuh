@@ -95,6 +95,7 @@ struct WsLayout {
     int64_t max_rows;
     int n_chunks;
     size_t planes, rowscale;   // E4M3 weights + bf16 activations only (else 0 bytes)
+    size_t tok_cnt;            // fused combine: arrival counters [T, ceil(H/128)], zeroed with ctrl
     int acc_cols;         // accumulator columns of the widest GEMM tile
 };
 
@@ -112,8 +113,9 @@ bool ws_layout(const moe_shape_t &s, WsLayout &L);
 int validate_shape(const moe_shape_t *s, bool need_gemm);
 
 // ---- launchers (return cudaError_t of the launch) ----
+// the first kernel of a layer call also clears n_zero words at `zero`
 cudaError_t launch_route(const moe_shape_t &s, const float *logits, int32_t *ids, float *w,
-                         cudaStream_t st);
+                         cudaStream_t st, int32_t *zero = nullptr, int n_zero = 0, bool chained = false);
 // router logits x . Wg^T and top-k in one launch; tickets [T] must be zero
 cudaError_t launch_router(const moe_shape_t &s, const void *x, const void *wg, float *logits,
                           int32_t *tickets, int32_t *ids, float *w, cudaStream_t st, bool chained);
@@ -126,9 +128,15 @@ cudaError_t launch_align(const moe_shape_t &s, const int32_t *ids, int32_t *coun
                          int32_t *offsets, int32_t *sorted_rows, int32_t *inv, int32_t *chunk_hist,
                          int32_t *chunk_base, Ctrl *ctrl, cudaStream_t st, int *launches,
                          bool chained = false, bool ticket_zero = false);
+// Routing + alignment of a batch with T*k <= 1024 routed rows in one block,
+// clearing the n_zero words at `zero` (status, ticket, tile and combine
+// counters) first.
+cudaError_t launch_route_align(const moe_shape_t &s, const float *logits, float *w, int32_t *counts,
+                               int32_t *offsets, int32_t *sorted_rows, int32_t *inv, Ctrl *ctrl, int32_t *zero,
+                               int n_zero, cudaStream_t st, bool chained);
 cudaError_t launch_gather(const moe_shape_t &s, const void *x, const int32_t *sorted_rows,
                           const int32_t *offsets, float a1, void *xp, int64_t max_rows,
-                          cudaStream_t st, bool chained = false);
+                          cudaStream_t st, bool chained = false, bool skip_pad = false);
 cudaError_t launch_combine(const moe_shape_t &s, const float *y, const float *w,
                            const int32_t *inv, const int32_t *offsets, void *out,
                            cudaStream_t st, bool chained = false);
@@ -136,9 +144,10 @@ cudaError_t launch_combine(const moe_shape_t &s, const float *y, const float *w,
 // Split bf16 rows [offsets[E+n_shared], K] of `src` into E4M3 planes hi
 // (rows 0..) and lo (rows max_rows..) of `planes` with v = scale[row] *
 // (hi + lo); see small_kernels.cu.
+// sorted_rows (may be NULL): skip the rows of pad slots
 cudaError_t launch_split_hilo(const moe_shape_t &s, const void *src, int K, const int32_t *offsets,
                               void *planes, float *scale, int64_t max_rows, cudaStream_t st,
-                              bool chained);
+                              bool chained, const int32_t *sorted_rows = nullptr);
 
 struct GemmArgs {
     int mode;                 // 0: gate/up + SwiGLU, 1: down projection
@@ -153,8 +162,17 @@ struct GemmArgs {
     float *partials;
     int64_t max_rows;
     bool chained;             // PDL launch; counters already zero
+    const int32_t *skip_pad_rows = nullptr;   // the layer's sorted_rows: pad slots' rows need no split
     void *planes;             // E4M3 weights + bf16 activations: hi/lo activation planes
     float *rowscale;          //   [2 * max_rows, K] E4M3 and the scale of each row
+    // fused combine (mode 1): slot -> row code; stage rows in ystage [T, k + n_shared, H],
+    // count them in tok_cnt [T, n_ct] (zero on entry), write out [T, H] bf16
+    bool combine = false;
+    const int32_t *sorted_rows = nullptr;
+    float *ystage = nullptr;
+    int32_t *tok_cnt = nullptr;
+    const float *wts = nullptr;
+    void *comb_out = nullptr;
 };
 cudaError_t launch_grouped_gemm(const moe_shape_t &s, const GemmPlan &p, const GemmArgs &a,
                                 cudaStream_t st, int *launches, int *host_err);

@@ -65,6 +65,20 @@ struct GemmParams {
                       // tiles are used throughout when the rounds are full enough:
                       // 1 (HBM-bound decode): >= 97% full on average;
                       // 2 (tensor-bound prefill): >= 90% full on average.
+    const int32_t *sorted_rows;   // slot -> row code (combine)
+    int T, k, R, n_shared;        // tokens, top-k, routed rows T*k, shared experts
+    // Fused combine (mode 1): instead of y in slot order, each row is staged
+    // as ystage[t][j] (row code f = t*k + j, or shared expert s as j = k + s)
+    // and counted per (token, output-feature tile); the CTA that brings a
+    // token's count to k + n_shared writes out[t] for that tile's features:
+    // sum_j w[t,j] * y[t,j] (fma, in j order) + sum_s y[t,k+s], rounded to
+    // bf16 -- the arithmetic and order of the separate combine step.
+    int combine;
+    float *ystage;
+    int32_t *tok_cnt;             // [T][n_ct], zero on entry
+    int n_ct;                     // output-feature tiles per token row
+    const float *wts;             // router weights [T, k]
+    __nv_bfloat16 *comb_out;      // out [T, H]
 };
 
 template <int kMode, bool kSwap, bool kFp8, int kBN, bool kHiLo = false, bool kPair = false>
@@ -265,6 +279,16 @@ __global__ void __launch_bounds__(Cfg<kMode, kSwap, kFp8, kBN, kHiLo, kPair>::kT
     // bank conflicts) so that the output is written as whole row segments
     constexpr int kStagePitch = 80;
     __shared__ __align__(16) uint8_t s_out_stage[kSwap ? 16 : C::kEpiWarps * 32 * kStagePitch];
+    // fused combine, per tile: each row's staging row and token, and the
+    // tokens this CTA finishes
+    constexpr int kTileRowsCta = kSwap ? kBN : 128;
+    __shared__ int s_dst[kMode == 1 ? kTileRowsCta : 1];
+    __shared__ int s_tok[kMode == 1 ? kTileRowsCta : 1];
+    __shared__ int s_fin[kMode == 1 ? kTileRowsCta : 1];
+    __shared__ int s_nfin;
+    // kPair tear-down: stage fills this CTA's producer issued, and the peer's
+    // fill count and abort flag (written by the peer)
+    __shared__ int s_fills, s_peer_fills, s_peer_abort;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int Et = p.E_tot;
@@ -277,6 +301,9 @@ __global__ void __launch_bounds__(Cfg<kMode, kSwap, kFp8, kBN, kHiLo, kPair>::kT
     // ---- set-up: barriers, tensor memory, tile table ----
     if (threadIdx.x == 0) {
         s_abort = 0;
+        s_fills = 0;
+        s_peer_fills = 0;
+        s_peer_abort = 0;
         for (int i = 0; i < C::kSlots; ++i) {
             mbar_init(smem_u32(&s_full[i]), 1);
             mbar_init(smem_u32(&s_empty[i]), 1);
@@ -474,10 +501,11 @@ __global__ void __launch_bounds__(Cfg<kMode, kSwap, kFp8, kBN, kHiLo, kPair>::kT
                     }
                 }
             }
+            s_fills = in_flight;
             if (!ok) {
                 // let issued copies land (kPair: rank 1's copies complete on rank
-                // 0's barriers; the pair waits out its copies at tear-down)
-                if (!kPair || rank == 0) drain_ring(s_full, n_stages, stage, phase, in_flight);
+                // 0's barriers; the pair retires its fills at tear-down)
+                if (!kPair) drain_ring(s_full, n_stages, stage, phase, in_flight);
             } else if (kPair) {
                 // every stage this CTA filled has been consumed, so no commit of
                 // rank 0's MMAs is still on its way to this CTA's barriers
@@ -577,7 +605,110 @@ __global__ void __launch_bounds__(Cfg<kMode, kSwap, kFp8, kBN, kHiLo, kPair>::kT
             // output scale of the tile; kHiLo: times the activation row's own
             // scale (column j of a Swap-AB tile is permuted row row0 + j)
             const float sc = (kHiLo ? 1.0f : p.ascale) * (p.wscale ? __ldg(&p.wscale[it.e]) : 1.0f);
+            // fused combine: each row's staging row and token (-1 for pad
+            // slots), a per-tile table filled by all epilogue threads before use
+            if constexpr (kMode == 1) {
+                for (int i = etid; p.combine && i < rows; i += C::kEpiThreads) {
+                    const int code = __ldg(p.sorted_rows + row0 + i);
+                    int t = -1, dst = -1;
+                    if (code >= 0) {
+                        const int kS = p.k + p.n_shared;
+                        if (code < p.R) {
+                            t = code / p.k;
+                            dst = t * kS + (code - t * p.k);
+                        } else {
+                            const int sh = (code - p.R) / p.T;
+                            t = code - p.R - sh * p.T;
+                            dst = t * kS + p.k + sh;
+                        }
+                    }
+                    s_dst[i] = dst;
+                    s_tok[i] = t;
+                }
+                if (p.combine) {
+                    if (etid == 0) s_nfin = 0;
+                    named_bar_sync(1, C::kEpiThreads);
+                }
+            }
+            // kHiLo: times the activation row's own scale (column j of a
+            // Swap-AB tile is permuted row row0 + j)
             auto col_sc = [&](int j) -> float { return kHiLo ? sc * __ldg(&p.rowscale[row0 + j]) : sc; };
+            // Fused combine, after this CTA has staged its rows of the tile:
+            // count each row in for (token, feature tile) and finish the tokens
+            // whose last row this was (output features [h0, h0 + fcols)).
+            // The staging stores of all epilogue threads are ordered before each
+            // arrival by the barrier and the arriving thread's fence; the
+            // finishing CTA's fence after its arrival orders its reads after
+            // every other CTA's stores.  The finishing work is spread over all
+            // epilogue threads as (token, 4 features) items, kU items per thread
+            // at a time with all their loads issued before any is used.
+            auto combine_tail = [&](int nrows, int h0, int fcols) {
+                named_bar_sync(1, C::kEpiThreads);
+                const int kS = p.k + p.n_shared;
+                for (int i = etid; i < nrows; i += C::kEpiThreads) {
+                    const int t = s_tok[i];
+                    if (t < 0) continue;
+                    __threadfence();
+                    if (atomicAdd(&p.tok_cnt[static_cast<size_t>(t) * p.n_ct + it.ft], 1) == kS - 1)
+                        s_fin[atomicAdd(&s_nfin, 1)] = t;
+                }
+                named_bar_sync(1, C::kEpiThreads);
+                const int nf = s_nfin;
+                if (nf == 0) return;
+                __threadfence();
+                const int ngrp = min(fcols, p.n_feat - h0) / 4;      // 4-feature groups
+                const int items = nf * ngrp;
+                // rows of a token prefetched per item (the rest load in order) and
+                // items per thread at a time: the 192-thread Swap-AB kernels have
+                // registers to spare, the 320-thread CTA-pair ones do not
+                constexpr int kU = 2;
+                constexpr int kMaxS = kSwap ? 9 : 4;
+                for (int base = etid; base < items; base += kU * C::kEpiThreads) {
+                    float4 v[kU][kMaxS];
+                    int tk[kU], g4[kU];
+#pragma unroll
+                    for (int u = 0; u < kU; ++u) {
+                        const int item = base + u * C::kEpiThreads;
+                        tk[u] = item < items ? s_fin[item / ngrp] : -1;
+                        g4[u] = item < items ? item % ngrp : 0;
+                        if (tk[u] < 0) continue;
+                        const float4 *yr = reinterpret_cast<const float4 *>(
+                            p.ystage + static_cast<size_t>(tk[u]) * kS * p.out_ld + h0 + 4 * g4[u]);
+#pragma unroll
+                        for (int j = 0; j < kMaxS; ++j)
+                            if (j < kS) v[u][j] = __ldcg(yr + static_cast<size_t>(j) * (p.out_ld / 4));
+                    }
+#pragma unroll
+                    for (int u = 0; u < kU; ++u) {
+                        if (tk[u] < 0) continue;
+                        const float4 *yr = reinterpret_cast<const float4 *>(
+                            p.ystage + static_cast<size_t>(tk[u]) * kS * p.out_ld + h0 + 4 * g4[u]);
+                        const float *wt = p.wts + static_cast<size_t>(tk[u]) * p.k;
+                        float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+                        // sum_j w_j y_j (fma, j order), then the shared rows
+                        auto add_row = [&](int j, const float4 &y) {
+                            if (j < p.k) {
+                                const float wj = __ldg(wt + j);
+                                a.x = fmaf(wj, y.x, a.x);
+                                a.y = fmaf(wj, y.y, a.y);
+                                a.z = fmaf(wj, y.z, a.z);
+                                a.w = fmaf(wj, y.w, a.w);
+                            } else {
+                                a.x += y.x;
+                                a.y += y.y;
+                                a.z += y.z;
+                                a.w += y.w;
+                            }
+                        };
+#pragma unroll
+                        for (int j = 0; j < kMaxS; ++j)
+                            if (j < kS) add_row(j, v[u][j]);
+                        for (int j = kMaxS; j < kS; ++j) add_row(j, __ldcg(yr + static_cast<size_t>(j) * (p.out_ld / 4)));
+                        *reinterpret_cast<uint2 *>(p.comb_out + static_cast<size_t>(tk[u]) * p.out_ld + h0 + 4 * g4[u]) =
+                            make_uint2(pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w));
+                    }
+                }
+            };
             const uint32_t tacc = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * C::kAccCols;
             // 16 accumulator columns starting at c0 (kHiLo: hi plane + lo plane)
             auto ld_acc16 = [&](int c0, uint32_t (&v)[16]) {
@@ -625,10 +756,19 @@ __global__ void __launch_bounds__(Cfg<kMode, kSwap, kFp8, kBN, kHiLo, kPair>::kT
                         uint32_t v[16];
                         ld_acc16(c0, v);
                         tmem_wait_ld();
+                        if (p.combine) {
 #pragma unroll
-                        for (int j = 0; j < 16; ++j)
-                            static_cast<float *>(p.out)[static_cast<size_t>(row0 + c0 + j) * p.out_ld + h0 + r] =
-                                __uint_as_float(v[j]) * col_sc(c0 + j);
+                            for (int j = 0; j < 16; ++j) {
+                                const int dr = s_dst[c0 + j];
+                                if (dr >= 0)
+                                    p.ystage[static_cast<size_t>(dr) * p.out_ld + h0 + r] = __uint_as_float(v[j]) * col_sc(c0 + j);
+                            }
+                        } else {
+#pragma unroll
+                            for (int j = 0; j < 16; ++j)
+                                static_cast<float *>(p.out)[static_cast<size_t>(row0 + c0 + j) * p.out_ld + h0 + r] =
+                                    __uint_as_float(v[j]) * col_sc(c0 + j);
+                        }
                     }
                 } else if (kMode == 0) {
                     // 32 features per chunk: h row segment of 64 (bf16) or 32 (E4M3) bytes
@@ -703,9 +843,13 @@ __global__ void __launch_bounds__(Cfg<kMode, kSwap, kFp8, kBN, kHiLo, kPair>::kT
                             const int rl = ps * 8 + (lane >> 2);
                             const int rg = q * 32 + rl;
                             const float4 val = *reinterpret_cast<const float4 *>(stg + rl * kStagePitch + (lane & 3) * 16);
-                            if (rg < rows)
-                                *reinterpret_cast<float4 *>(static_cast<float *>(p.out) +
-                                                            static_cast<size_t>(row0 + rg) * p.out_ld + h0 + c0 + (lane & 3) * 4) = val;
+                            if (rg < rows) {
+                                const int dr = p.combine ? s_dst[rg] : row0 + rg;
+                                float *dstp = p.combine ? p.ystage : static_cast<float *>(p.out);
+                                if (dr >= 0)
+                                    *reinterpret_cast<float4 *>(dstp + static_cast<size_t>(dr) * p.out_ld + h0 + c0 + (lane & 3) * 4) =
+                                        val;
+                            }
                         }
                         __syncwarp();
                     }
@@ -717,6 +861,8 @@ __global__ void __launch_bounds__(Cfg<kMode, kSwap, kFp8, kBN, kHiLo, kPair>::kT
                     if constexpr (kPair) mbar_arrive_cluster(mapa_shared(smem_u32(&s_tempty[acc]), 0));
                     else mbar_arrive(smem_u32(&s_tempty[acc]));
                 }
+                if constexpr (kMode == 1)
+                    if (p.combine) combine_tail(rows, it.ft * (kSwap ? 128 : 256), kSwap ? 128 : 256);
             } else {
                 // ---- one share of a split tile: store the raw partial ----
                 float *slot = p.partials + static_cast<size_t>(it.slot) * 128 * C::kAccCols;
@@ -773,8 +919,13 @@ __global__ void __launch_bounds__(Cfg<kMode, kSwap, kFp8, kBN, kHiLo, kPair>::kT
                         for (int j = 0; j < ncols; ++j) {
                             float a = 0.f;
                             for (int c = c_first; c <= c_last; ++c) a += __ldcg(&slot_of(c)[j * 128 + etid]);
-                            static_cast<float *>(p.out)[static_cast<size_t>(row0 + j) * p.out_ld + h0 + etid] = a * col_sc(j);
+                            if (!p.combine)
+                                static_cast<float *>(p.out)[static_cast<size_t>(row0 + j) * p.out_ld + h0 + etid] = a * col_sc(j);
+                            else if (s_dst[j] >= 0)
+                                p.ystage[static_cast<size_t>(s_dst[j]) * p.out_ld + h0 + etid] = a * col_sc(j);
                         }
+                        if constexpr (kMode == 1)
+                            if (p.combine) combine_tail(ncols, h0, 128);
                     } else if (kMode == 0) {
                         const int f0 = it.ft * 128;
                         const int rr = etid & 127, hf = etid >> 7;
@@ -794,12 +945,16 @@ __global__ void __launch_bounds__(Cfg<kMode, kSwap, kFp8, kBN, kHiLo, kPair>::kT
                     } else {
                         const int h0 = it.ft * 256;
                         const int rr = etid & 127, hf = etid >> 7;
-                        if (rr < rows)
+                        const int dr = rr < rows ? (p.combine ? s_dst[rr] : row0 + rr) : -1;
+                        float *dstp = p.combine ? p.ystage : static_cast<float *>(p.out);
+                        if (dr >= 0)
                             for (int j = hf * (256 / kNch); j < (hf + 1) * (256 / kNch) && h0 + j < p.n_feat; ++j) {
                                 float a = 0.f;
                                 for (int c = c_first; c <= c_last; ++c) a += __ldcg(&slot_of(c)[j * 128 + rr]);
-                                static_cast<float *>(p.out)[static_cast<size_t>(row0 + rr) * p.out_ld + h0 + j] = a * sc;
+                                dstp[static_cast<size_t>(dr) * p.out_ld + h0 + j] = a * sc;
                             }
+                        if constexpr (kMode == 1)
+                            if (p.combine) combine_tail(rows, h0, 256);
                     }
                 }
                 named_bar_sync(1, C::kEpiThreads);
@@ -815,14 +970,33 @@ __global__ void __launch_bounds__(Cfg<kMode, kSwap, kFp8, kBN, kHiLo, kPair>::kT
     tc_fence_before();
     __syncthreads();
     if constexpr (kPair) {
-        // After an abort, copies issued by this CTA may still be landing in its
-        // shared memory (their completion was signalled to rank 0): give them
-        // time.  Then neither CTA leaves while the other may still signal it.
-        if (s_abort) {
-            const uint64_t t0 = globaltimer();
-            while (globaltimer() - t0 < 200000ull) {}
+        // Each CTA tells the other how many stage fills it issued and whether
+        // it aborted; neither leaves while the other may still signal it.
+        if (threadIdx.x == 0) {
+            st_shared_cluster(mapa_shared(smem_u32(&s_peer_fills), rank ^ 1u), static_cast<uint32_t>(s_fills));
+            st_shared_cluster(mapa_shared(smem_u32(&s_peer_abort), rank ^ 1u), static_cast<uint32_t>(s_abort));
         }
         cluster_sync();
+        if (s_abort || s_peer_abort) {                  // the same decision in both CTAs
+            // After an abort some copies may still be landing.  Both CTAs' halves
+            // of fill i complete on rank 0's full barrier of stage i % n_stages,
+            // in phase (i / n_stages) & 1.  Rank 0 retires the last ring's worth
+            // of fills: a fill only rank 1 issued is armed for its half, a fill
+            // only rank 0 issued gets rank 1's half counted as done, then every
+            // phase is awaited (bounded), so no copy into either CTA is in flight
+            // when they leave.  Older fills were consumed by the MMAs already.
+            if (rank == 0 && threadIdx.x == 0) {
+                const int n0 = s_fills, n1 = s_peer_fills, nmax = max(n0, n1);
+                for (int i = max(0, nmax - n_stages); i < nmax; ++i) {
+                    const uint32_t fb = smem_u32(&s_full[i % n_stages]);
+                    if (i >= n0) mbar_arrive_expect_tx(fb, C::kStage);
+                    else if (i >= n1) mbar_complete_tx(fb, C::kStage);
+                    volatile int no_abort = 0;
+                    mbar_wait(fb, static_cast<uint32_t>((i / n_stages) & 1), &no_abort);
+                }
+            }
+            cluster_sync();
+        }
     }
     if (threadIdx.x == 0 && s_abort) set_status(p.status, MOE_ERR_TIMEOUT);
     if (warp == 1) {
@@ -853,10 +1027,30 @@ static EncodeTiledFn get_encode_fn()
 }
 
 // 2-D map over a row-major [rows, cols] matrix with 128-byte rows per box
-// and the 128-byte swizzle; box = box_rows x (128 bytes).
+// and the 128-byte swizzle; box = box_rows x (128 bytes).  A map depends only
+// on these arguments (not on the device or on what the memory holds), so the
+// last few are kept per host thread and a repeat call with the same buffers
+// skips the encode.
 static bool make_map(CUtensorMap *m, const void *base, bool u8, uint64_t rows, uint64_t cols,
                      uint32_t box_rows)
 {
+    struct Entry {
+        const void *base;
+        uint64_t rows, cols;
+        uint32_t box_rows;
+        bool u8, valid;
+        CUtensorMap map;
+    };
+    constexpr int kEntries = 16;
+    thread_local Entry cache[kEntries] = {};
+    thread_local int next = 0;
+    for (int i = 0; i < kEntries; ++i) {
+        const Entry &c = cache[i];
+        if (c.valid && c.base == base && c.rows == rows && c.cols == cols && c.box_rows == box_rows && c.u8 == u8) {
+            *m = c.map;
+            return true;
+        }
+    }
     constexpr uint32_t row_bytes = 128;
     EncodeTiledFn fn = get_encode_fn();
     if (!fn) return false;
@@ -870,7 +1064,11 @@ static bool make_map(CUtensorMap *m, const void *base, bool u8, uint64_t rows, u
                     CU_TENSOR_MAP_SWIZZLE_128B,
                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS;
+    if (r != CUDA_SUCCESS) return false;
+    Entry &c = cache[next];
+    next = (next + 1) % kEntries;
+    c = Entry{base, rows, cols, box_rows, u8, true, *m};
+    return true;
 }
 
 // SMs of the current device (the persistent grid size), cached per device.
@@ -961,6 +1159,17 @@ static cudaError_t run_gemm(const moe_shape_t &s, const GemmArgs &a, cudaStream_
     p.partials = a.partials;
     p.rowscale = a.rowscale;
     p.lo_rows = static_cast<int>(a.max_rows);
+    p.sorted_rows = a.sorted_rows;
+    p.T = s.T;
+    p.k = s.k;
+    p.R = s.T * s.k;
+    p.n_shared = s.n_shared;
+    p.combine = kMode == 1 && a.combine ? 1 : 0;
+    p.ystage = a.ystage;
+    p.tok_cnt = a.tok_cnt;
+    p.n_ct = (s.H + (kSwap ? 127 : 255)) / (kSwap ? 128 : 256);
+    p.wts = a.wts;
+    p.comb_out = static_cast<__nv_bfloat16 *>(a.comb_out);
     // decode tiles split cheaply (few token columns); prefill tiles carry
     // 128 KB of fp32 partials, so whole tiles are preferred there; CTA pairs
     // take whole tiles only
@@ -1008,7 +1217,7 @@ cudaError_t launch_grouped_gemm(const moe_shape_t &s, const GemmPlan &p, const G
             if (err != cudaSuccess) return err;
         }
         err = launch_split_hilo(s, a.act, a.mode == 0 ? s.H : s.I, a.offsets, a.planes, a.rowscale,
-                                a.max_rows, st, a.chained);
+                                a.max_rows, st, a.chained, a.skip_pad_rows);
         if (err != cudaSuccess) return err;
         *launches += 1;
         GemmArgs g = a;

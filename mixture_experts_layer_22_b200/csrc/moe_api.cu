@@ -80,7 +80,9 @@ bool ws_layout(const moe_shape_t &s, WsLayout &L)
     // stream-K tile counters right after the control words (one memset
     // clears both): GEMM1 uses the first half, GEMM2 the second
     L.counters = o;    o += up256(4 * kMaxCtas * 4);
-    // router tickets, also cleared by that memset
+    // the fused combine's arrival counters per (token, 128-feature tile), then
+    // the router tickets: all cleared together with the control words
+    L.tok_cnt = o;     o += up256(static_cast<size_t>(s.T) * ((s.H + 127) / 128) * 4);
     L.tickets = o;     o += up256(static_cast<size_t>(s.T) * 4);
     L.logits = o;      o += up256(static_cast<size_t>(s.T) * s.E * 4);
     L.ids = o;         o += up256(R * 4);
@@ -93,7 +95,8 @@ bool ws_layout(const moe_shape_t &s, WsLayout &L)
     L.inv = o;         o += up256(R * 4);
     L.xp = o;          o += up256(L.max_rows * s.H * ab);
     L.h = o;           o += up256(L.max_rows * s.I * ab);
-    L.y = o;           o += up256(L.max_rows * s.H * 4);
+    // fused combine: down-projection rows staged per (token, choice) [T, k+S, H] fp32
+    L.y = o;           o += up256(static_cast<size_t>(s.T) * (s.k + s.n_shared) * s.H * 4);
     L.partials = o;    o += up256(static_cast<size_t>(2 * kMaxCtas) * 128 * L.acc_cols * 4);
     // hi/lo E4M3 planes of GEMM1's then GEMM2's activations (reused: the
     // split of h runs after GEMM1 has finished reading the planes of xp)
@@ -318,23 +321,39 @@ static int fused_impl(const moe_shape_t *shape, const void *x, const float *logi
     void *h = b + L.h;
     float *y = reinterpret_cast<float *>(b + L.y);
 
-    // One memset clears the status, the align ticket, both GEMMs' tile
-    // counters and the router's tickets (adjacent in the workspace).  Every
-    // later kernel is a programmatic dependent launch of the one before it,
-    // so there is no other non-kernel node in the sequence.
-    cudaError_t e = cudaMemsetAsync(ctrl, 0, L.tickets + static_cast<size_t>(s.T) * sizeof(int32_t) - L.ctrl, sm);
-    if (e != cudaSuccess) return MOE_ERR_CUDA;
-    if (wg)
-        e = launch_router(s, x, wg, reinterpret_cast<float *>(b + L.logits),
-                          reinterpret_cast<int32_t *>(b + L.tickets), ids, w, sm, false);
-    else
-        e = launch_route(s, logits, ids, w, sm);
-    if (e != cudaSuccess) return MOE_ERR_CUDA;
-    g_launches += 1;
-    e = launch_align(s, ids, counts, offsets, rows, inv, reinterpret_cast<int32_t *>(b + L.chunk_hist),
-                     reinterpret_cast<int32_t *>(b + L.chunk_base), ctrl, sm, &g_launches, true);
-    if (e != cudaSuccess) return MOE_ERR_CUDA;
-    e = launch_gather(s, x, rows, offsets, a1_scale, xp, L.max_rows, sm, true);
+    cudaError_t e;
+    const int n_zero = static_cast<int>((L.tickets - L.ctrl) / sizeof(int32_t));
+    if (!wg && s.T <= 32 && static_cast<int64_t>(s.T) * s.k <= kAlignChunk) {
+        // A small decode batch (a warp per token): routing and alignment in one block, which first
+        // clears the status, the align ticket and both GEMMs' tile counters
+        // (adjacent at the start of the workspace).  It is a programmatic
+        // dependent launch like every kernel after it: it waits for whatever
+        // ran before it on the stream before touching the workspace.
+        e = launch_route_align(s, logits, w, counts, offsets, rows, inv, ctrl, reinterpret_cast<int32_t *>(ctrl),
+                               n_zero, sm, true);
+        if (e != cudaSuccess) return MOE_ERR_CUDA;
+        g_launches += 1;
+    } else {
+        if (wg) {
+            // the router kernel counts per-token tickets: one memset clears
+            // them with the control words and counters (adjacent)
+            e = cudaMemsetAsync(ctrl, 0, L.tickets + static_cast<size_t>(s.T) * sizeof(int32_t) - L.ctrl, sm);
+            if (e != cudaSuccess) return MOE_ERR_CUDA;
+            e = launch_router(s, x, wg, reinterpret_cast<float *>(b + L.logits),
+                              reinterpret_cast<int32_t *>(b + L.tickets), ids, w, sm, false);
+        } else {
+            // the route kernel (a warp per token) clears the control words and
+            // counters itself; like every kernel after it, it is a programmatic
+            // dependent launch that waits for the stream's earlier work first
+            e = launch_route(s, logits, ids, w, sm, reinterpret_cast<int32_t *>(ctrl), n_zero, true);
+        }
+        if (e != cudaSuccess) return MOE_ERR_CUDA;
+        g_launches += 1;
+        e = launch_align(s, ids, counts, offsets, rows, inv, reinterpret_cast<int32_t *>(b + L.chunk_hist),
+                         reinterpret_cast<int32_t *>(b + L.chunk_base), ctrl, sm, &g_launches, true);
+        if (e != cudaSuccess) return MOE_ERR_CUDA;
+    }
+    e = launch_gather(s, x, rows, offsets, a1_scale, xp, L.max_rows, sm, true, true);
     if (e != cudaSuccess) return MOE_ERR_CUDA;
     g_launches += 1;
     const GemmPlan plan = plan_gemm(s);
@@ -347,6 +366,7 @@ static int fused_impl(const moe_shape_t *shape, const void *x, const float *logi
     a.rowscale = reinterpret_cast<float *>(b + L.rowscale);
     a.max_rows = L.max_rows;
     a.offsets = offsets;
+    a.skip_pad_rows = rows;
     int host_err = MOE_OK;
     a.mode = 0;
     a.act = xp;
@@ -358,19 +378,23 @@ static int fused_impl(const moe_shape_t *shape, const void *x, const float *logi
     e = launch_grouped_gemm(s, plan, a, sm, &g_launches, &host_err);
     if (host_err != MOE_OK) return host_err;
     if (e != cudaSuccess) return MOE_ERR_CUDA;
+    // GEMM2 with the combine fused into its epilogue: out is written there
     a.mode = 1;
     a.act = h;
     a.wgt = w2;
     a.wscale = w2_scale;
     a.ascale = s.adtype == MOE_E4M3 ? a2_scale : 1.0f;
     a.out = y;
+    a.combine = true;
+    a.sorted_rows = rows;
+    a.ystage = y;
+    a.tok_cnt = reinterpret_cast<int32_t *>(b + L.tok_cnt);
+    a.wts = w;
+    a.comb_out = out;
     a.counters += 2 * kMaxCtas;
     e = launch_grouped_gemm(s, plan, a, sm, &g_launches, &host_err);
     if (host_err != MOE_OK) return host_err;
     if (e != cudaSuccess) return MOE_ERR_CUDA;
-    e = launch_combine(s, y, w, inv, offsets, out, sm, true);
-    if (e != cudaSuccess) return MOE_ERR_CUDA;
-    g_launches += 1;
     return MOE_OK;
 }
 

@@ -103,6 +103,20 @@ __device__ __forceinline__ void cluster_sync()
                      "memory");
 }
 
+// Store a 32-bit value into the shared memory of a CTA of the cluster
+// (shared::cluster address from mapa_shared).
+__device__ __forceinline__ void st_shared_cluster(uint32_t addr_cluster, uint32_t v)
+{
+    asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(addr_cluster), "r"(v) : "memory");
+}
+
+// Count `bytes` of the barrier's current phase as arrived, as if a copy had
+// delivered them (used to retire a phase whose copies were never issued).
+__device__ __forceinline__ void mbar_complete_tx(uint32_t bar, uint32_t bytes)
+{
+    asm volatile("mbarrier.complete_tx.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+
 // Arrive on an mbarrier that may live in the peer CTA (shared::cluster address).
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar_cluster)
 {

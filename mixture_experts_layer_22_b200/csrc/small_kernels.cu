@@ -100,15 +100,18 @@ __device__ __forceinline__ void route_warp(const float *l, int E, int k, int gat
     }
 }
 
-// One warp per token.
+// One warp per token.  As the first kernel of the fused layer it also clears
+// `n_zero` words at `zero` (the control words and counters the later kernels
+// use after their dependency waits); nothing in this kernel reads them.
 template <int kSlots>
 __global__ void __launch_bounds__(256) route_topk_kernel(const float *__restrict__ logits, int T,
                                                          int E, int k, int gate, int renorm,
                                                          float routed_scale, int32_t *ids,
-                                                         float *w)
+                                                         float *w, int32_t *zero, int n_zero)
 {
     grid_dep_wait();
     grid_dep_launch();
+    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n_zero; i += gridDim.x * blockDim.x) zero[i] = 0;
     const int lane = threadIdx.x & 31;
     const int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     if (t >= T) return;
@@ -117,20 +120,19 @@ __global__ void __launch_bounds__(256) route_topk_kernel(const float *__restrict
 }
 
 cudaError_t launch_route(const moe_shape_t &s, const float *logits, int32_t *ids, float *w,
-                         cudaStream_t st)
+                         cudaStream_t st, int32_t *zero, int n_zero, bool chained)
 {
     const int threads = 256, blocks = (s.T * 32 + threads - 1) / threads;
     const int slots = (s.E + 31) / 32;
-#define MOE_ROUTE(N)                                                                          \
-    route_topk_kernel<N><<<blocks, threads, 0, st>>>(logits, s.T, s.E, s.k, s.gate, s.renorm, \
-                                                     s.routed_scale, ids, w)
+#define MOE_ROUTE(N)                                                                                            \
+    return launch_kernel(route_topk_kernel<N>, dim3(blocks), dim3(threads), 0, st, chained, logits, s.T, s.E, s.k, \
+                         s.gate, s.renorm, s.routed_scale, ids, w, zero, n_zero)
     if (slots <= 1) MOE_ROUTE(1);
-    else if (slots <= 2) MOE_ROUTE(2);
-    else if (slots <= 4) MOE_ROUTE(4);
-    else if (slots <= 8) MOE_ROUTE(8);
-    else MOE_ROUTE(16);
+    if (slots <= 2) MOE_ROUTE(2);
+    if (slots <= 4) MOE_ROUTE(4);
+    if (slots <= 8) MOE_ROUTE(8);
+    MOE_ROUTE(16);
 #undef MOE_ROUTE
-    return cudaGetLastError();
 }
 
 // ------------------------------------------------------------------ router
@@ -355,16 +357,13 @@ __global__ void __launch_bounds__(1024) align_scatter_kernel(const int32_t *__re
 }
 
 // All routed rows in one block (R <= 1024, every decode batch here): count,
-// scan, pad and place in a single launch, with the histogram, the offsets and
-// the per-warp counts in shared memory.  Same result as the two-kernel path.
-__global__ void __launch_bounds__(1024) align_single_kernel(const int32_t *__restrict__ ids, int R, int T,
-                                                            int E, int n_shared, int pad, int32_t *counts,
-                                                            int32_t *offsets, int32_t *sorted_rows,
-                                                            int32_t *inv, Ctrl *ctrl)
+// scan, pad and place, with the histogram, the offsets and the per-warp counts
+// in shared memory sm_al [33 * Et].  Same result as the two-kernel path.
+// `ids` may live in global or shared memory; the whole block calls this.
+__device__ __forceinline__ void align_block(const int32_t *ids, int R, int T, int E, int n_shared, int pad,
+                                            int32_t *counts, int32_t *offsets, int32_t *sorted_rows,
+                                            int32_t *inv, Ctrl *ctrl, int32_t *sm_al)
 {
-    grid_dep_wait();
-    grid_dep_launch();
-    extern __shared__ int32_t sm_al[];
     const int Et = E + n_shared;
     int32_t *hist = sm_al;                 // [Et]: counts, then segment starts
     int32_t *wc = sm_al + Et;              // [32 warps][Et]
@@ -434,6 +433,72 @@ __global__ void __launch_bounds__(1024) align_single_kernel(const int32_t *__res
     }
 }
 
+__global__ void __launch_bounds__(1024) align_single_kernel(const int32_t *__restrict__ ids, int R, int T,
+                                                            int E, int n_shared, int pad, int32_t *counts,
+                                                            int32_t *offsets, int32_t *sorted_rows,
+                                                            int32_t *inv, Ctrl *ctrl)
+{
+    grid_dep_wait();
+    grid_dep_launch();
+    extern __shared__ int32_t sm_al[];
+    align_block(ids, R, T, E, n_shared, pad, counts, offsets, sorted_rows, inv, ctrl, sm_al);
+}
+
+// Routing and alignment of a decode batch in one block (R = T*k <= 1024), the
+// first kernel of the fused layer: it also clears the status word, the align
+// ticket, the GEMMs' stream-K tile counters and the fused combine's arrival
+// counters (`zero`, `n_zero` words), which the later kernels of the call use
+// only after their dependency waits.  Warp w
+// routes tokens w, w + 32, ... (as route_topk_kernel); the ids stay in shared
+// memory for the alignment.
+template <int kSlots>
+__global__ void __launch_bounds__(1024) route_align_kernel(const float *__restrict__ logits, int T, int E, int k,
+                                                           int gate, int renorm, float routed_scale, int n_shared,
+                                                           int pad, float *w, int32_t *counts, int32_t *offsets,
+                                                           int32_t *sorted_rows, int32_t *inv, Ctrl *ctrl,
+                                                           int32_t *zero, int n_zero)
+{
+    grid_dep_wait();
+    grid_dep_launch();
+    __shared__ int32_t s_ids[kAlignChunk];
+    extern __shared__ int32_t sm_al[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    for (int i = threadIdx.x; i < n_zero; i += blockDim.x) zero[i] = 0;
+    __syncthreads();                                     // status cleared before anything can set it
+    for (int t = warp; t < T; t += blockDim.x >> 5)
+        route_warp<kSlots>(logits + static_cast<size_t>(t) * E, E, k, gate, renorm, routed_scale, s_ids + t * k,
+                           w + static_cast<size_t>(t) * k, lane);
+    __syncthreads();
+    align_block(s_ids, T * k, T, E, n_shared, pad, counts, offsets, sorted_rows, inv, ctrl, sm_al);
+}
+
+cudaError_t launch_route_align(const moe_shape_t &s, const float *logits, float *w, int32_t *counts,
+                               int32_t *offsets, int32_t *sorted_rows, int32_t *inv, Ctrl *ctrl, int32_t *zero,
+                               int n_zero, cudaStream_t st, bool chained)
+{
+    const int Et = s.E + s.n_shared;
+    const int slots = (s.E + 31) / 32;
+    static PerDeviceOnce attrs;
+    attrs([] {
+        cudaFuncSetAttribute(route_align_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, 33 * kMaxExpertsTotal * 4);
+        cudaFuncSetAttribute(route_align_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, 33 * kMaxExpertsTotal * 4);
+        cudaFuncSetAttribute(route_align_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, 33 * kMaxExpertsTotal * 4);
+        cudaFuncSetAttribute(route_align_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, 33 * kMaxExpertsTotal * 4);
+        cudaFuncSetAttribute(route_align_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize, 33 * kMaxExpertsTotal * 4);
+    });
+    const size_t smem = 33 * Et * sizeof(int32_t);
+#define MOE_RA(N)                                                                                                  \
+    return launch_kernel(route_align_kernel<N>, dim3(1), dim3(kAlignChunk), smem, st, chained, logits, s.T, s.E, \
+                         s.k, s.gate, s.renorm, s.routed_scale, s.n_shared, s.pad, w, counts, offsets, sorted_rows, \
+                         inv, ctrl, zero, n_zero)
+    if (slots <= 1) MOE_RA(1);
+    if (slots <= 2) MOE_RA(2);
+    if (slots <= 4) MOE_RA(4);
+    if (slots <= 8) MOE_RA(8);
+    MOE_RA(16);
+#undef MOE_RA
+}
+
 cudaError_t launch_align(const moe_shape_t &s, const int32_t *ids, int32_t *counts,
                          int32_t *offsets, int32_t *sorted_rows, int32_t *inv, int32_t *chunk_hist,
                          int32_t *chunk_base, Ctrl *ctrl, cudaStream_t st, int *launches, bool chained,
@@ -469,11 +534,14 @@ cudaError_t launch_align(const moe_shape_t &s, const int32_t *ids, int32_t *coun
 
 // ------------------------------------------------------------------ gather
 // One warp per slot of the permuted buffer, 16-byte vectors along the row.
+// skip_pad: leave pad slots unwritten (inside the fused layer, where a pad
+// slot's row reaches no real output: an MMA column depends only on its own
+// operand row, and the combine skips pad slots); else write zeros there.
 template <bool kQuant>
 __global__ void __launch_bounds__(256) gather_kernel(const uint4 *__restrict__ x,
                                                      const int32_t *__restrict__ sorted_rows,
                                                      const int32_t *__restrict__ offsets, int Et,
-                                                     int T, int k, int H, float a1, void *xp)
+                                                     int T, int k, int H, float a1, void *xp, int skip_pad)
 {
     grid_dep_wait();
     grid_dep_launch();
@@ -488,7 +556,7 @@ __global__ void __launch_bounds__(256) gather_kernel(const uint4 *__restrict__ x
         const int v = static_cast<int>(item % nchunk) * 32 + lane;
         const int f = sorted_rows[s];
         const int t = f < 0 ? -1 : (f < R ? f / k : (f - R) % T);
-        if (v >= nvec) continue;
+        if (v >= nvec || (t < 0 && skip_pad)) continue;
         if (!kQuant) {
             uint4 *dst = reinterpret_cast<uint4 *>(xp) + static_cast<size_t>(s) * nvec;
             const uint4 *src = x + static_cast<size_t>(t < 0 ? 0 : t) * nvec;
@@ -517,7 +585,7 @@ __global__ void __launch_bounds__(256) gather_kernel(const uint4 *__restrict__ x
 
 cudaError_t launch_gather(const moe_shape_t &s, const void *x, const int32_t *sorted_rows,
                           const int32_t *offsets, float a1, void *xp, int64_t max_rows,
-                          cudaStream_t st, bool chained)
+                          cudaStream_t st, bool chained, bool skip_pad)
 {
     const int Et = s.E + s.n_shared;
     const int64_t warps = max_rows * ((s.H / 8 + 31) / 32);
@@ -526,7 +594,7 @@ cudaError_t launch_gather(const moe_shape_t &s, const void *x, const int32_t *so
     if (blocks < 1) blocks = 1;
     return launch_kernel(s.adtype == MOE_E4M3 ? gather_kernel<true> : gather_kernel<false>, dim3(blocks),
                          dim3(256), 0, st, chained, static_cast<const uint4 *>(x), sorted_rows, offsets, Et,
-                         s.T, s.k, s.H, a1, xp);
+                         s.T, s.k, s.H, a1, xp, skip_pad ? 1 : 0);
 }
 
 // ------------------------------------------------------------------ hi/lo split
@@ -588,10 +656,13 @@ __device__ __forceinline__ int row_scale_exp(float amax)
     return e < -126 ? -126 : e;
 }
 
-// One block per permuted row (grid-stride over the rows that exist).
+// One block per permuted row (grid-stride over the rows that exist).  With
+// sorted_rows (inside the fused layer) pad slots are skipped: their rows
+// reach no real output.
 __global__ void __launch_bounds__(256) split_hilo_kernel(const uint4 *__restrict__ src, int K,
                                                          const int32_t *__restrict__ offsets, int Et,
-                                                         int64_t lo_rows, uint2 *planes, float *scale)
+                                                         int64_t lo_rows, uint2 *planes, float *scale,
+                                                         const int32_t *__restrict__ sorted_rows)
 {
     grid_dep_wait();
     grid_dep_launch();
@@ -600,6 +671,7 @@ __global__ void __launch_bounds__(256) split_hilo_kernel(const uint4 *__restrict
     const int nv = K / 8;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     for (int row = blockIdx.x; row < total; row += gridDim.x) {
+        if (sorted_rows && sorted_rows[row] < 0) continue;       // the same for the whole block
         const uint4 *r = src + static_cast<size_t>(row) * nv;
         float m = 0.0f;
         for (int v = threadIdx.x; v < nv; v += blockDim.x) m = fmaxf(m, abs_max8(r[v]));
@@ -625,13 +697,14 @@ __global__ void __launch_bounds__(256) split_hilo_kernel(const uint4 *__restrict
 }
 
 cudaError_t launch_split_hilo(const moe_shape_t &s, const void *src, int K, const int32_t *offsets,
-                              void *planes, float *scale, int64_t max_rows, cudaStream_t st, bool chained)
+                              void *planes, float *scale, int64_t max_rows, cudaStream_t st, bool chained,
+                              const int32_t *sorted_rows)
 {
     int blocks = static_cast<int>(max_rows < 148 * 8 ? max_rows : 148 * 8);
     if (blocks < 1) blocks = 1;
     return launch_kernel(split_hilo_kernel, dim3(blocks), dim3(256), 0, st, chained,
                          static_cast<const uint4 *>(src), K, offsets, s.E + s.n_shared, max_rows,
-                         static_cast<uint2 *>(planes), scale);
+                         static_cast<uint2 *>(planes), scale, sorted_rows);
 }
 
 // ------------------------------------------------------------------ combine

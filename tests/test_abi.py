@@ -117,3 +117,26 @@ def test_misaligned_pointers_rejected(lib):
     assert r == -1
     r = lib.moe_fused_forward(C.byref(s), 256, 256, 256, None, 256, None, 1.0, 1.0, 256, 272, need, None)
     assert r == -1
+
+
+def _rope(**kw):
+    base = dict(num_tokens=8, n_heads=4, head_dim=128, rot_dim=128, max_pos=64, interleaved=0)
+    base.update(kw)
+    return moe.RopeShape(**base)
+
+
+@pytest.mark.parametrize("kw,code", [({"head_dim": 96, "rot_dim": 96}, -2), ({"rot_dim": 7}, -1),
+                                     ({"rot_dim": 24}, -2), ({"rot_dim": 24, "interleaved": 1, "num_tokens": 0}, 0),
+                                     ({"rot_dim": 130}, -1), ({"n_heads": 0}, -1), ({"interleaved": 2}, -1),
+                                     ({"num_tokens": -1}, -1), ({"max_pos": 0}, -1)])
+def test_inv_rope_rejects_bad_shapes_before_launch(lib, kw, code):
+    assert lib.moe_inv_rope_quant_per_head(C.byref(_rope(**kw)), 16, 16, 16, 16, 16, None, None) == code
+
+
+def test_inv_rope_rejects_null_and_misaligned_pointers(lib):
+    s = _rope()
+    assert lib.moe_inv_rope_quant_per_head(C.byref(s), None, 16, 16, 16, 16, None, None) == -1
+    assert lib.moe_inv_rope_quant_per_head(C.byref(s), 8, 16, 16, 16, 16, None, None) == -1   # x not 16-aligned
+    assert lib.moe_inv_rope_quant_per_head(C.byref(s), 16, 16, 16, 4, 16, None, None) == -1   # q not 8-aligned
+    assert lib.moe_inv_rope_quant_per_head(C.byref(_rope(num_tokens=0)), None, None, None, None, None, None,
+                                           None) == 0                                        # nothing to do

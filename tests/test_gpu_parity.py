@@ -477,3 +477,72 @@ def test_bounded_wait_times_out_and_context_stays_usable():
     got = L.run()                      # resets the status, runs the layer
     assert L.status() == 0
     assert rel_err(got, oracle_forward(wl, d), "bf16") <= BF16_TOL
+
+
+# ------------------------------------------------------------------ fused gather and combine
+# The fused layer gathers GEMM1's token rows straight from x (tile::gather4)
+# and combines inside GEMM2's epilogue.  The arithmetic and its order are
+# those of the separate steps, so the fused output must equal, bit for bit,
+# the output of the step-by-step calls on the same inputs.
+STEPWISE = [
+    (W["tiny"], moe.SWAP_AB), (W["tiny"], moe.NORMAL),
+    (EDGE[0], moe.SWAP_AB), (EDGE[0], moe.NORMAL),                  # ragged T=37
+    (EDGE[2], moe.AUTO),                                              # E=256 top-8 sigmoid + shared
+    (EDGE[3], moe.NORMAL),                                            # T=600 prefill, CTA-pair GEMM2
+    (EDGE[4], moe.SWAP_AB), (EDGE[4], moe.NORMAL),                   # T=300: several row tiles
+    (syn.Workload("fp8_small", T=300, H=512, I=512, E=8, k=2, wdtype=syn.E4M3, adtype=syn.E4M3, seed=7),
+     moe.SWAP_AB),
+    (syn.Workload("fp8_small", T=300, H=512, I=512, E=8, k=2, wdtype=syn.E4M3, adtype=syn.E4M3, seed=7),
+     moe.NORMAL),
+    (syn.Workload("dsv3_small", T=8, H=1024, I=256, E=256, k=8, n_shared=1, gate=syn.SIGMOID,
+                  routed_scale=2.5, wdtype=syn.E4M3, seed=8), moe.AUTO),
+    (syn.Workload("dsv3_small", T=128, H=1024, I=256, E=256, k=8, n_shared=1, gate=syn.SIGMOID,
+                  routed_scale=2.5, wdtype=syn.E4M3, seed=8), moe.AUTO),
+]
+
+
+def _stepwise(L, a2):
+    """The layer as separate entry-point calls (the unfused reference)."""
+    wl, s = L.wl, L.shape
+    E_t = wl.E + wl.n_shared
+    mr = moe.max_rows(s)
+    fp8a = wl.adtype == syn.E4M3
+    ids = torch.empty((wl.T, wl.k), dtype=torch.int32, device="cuda")
+    w = torch.empty((wl.T, wl.k), dtype=torch.float32, device="cuda")
+    counts = torch.empty(E_t, dtype=torch.int32, device="cuda")
+    offsets = torch.empty(E_t + 1, dtype=torch.int32, device="cuda")
+    rows = torch.empty(mr, dtype=torch.int32, device="cuda")
+    inv = torch.empty(wl.T * wl.k, dtype=torch.int32, device="cuda")
+    xp = torch.empty((mr, wl.H * (1 if fp8a else 2)), dtype=torch.uint8, device="cuda")
+    h = torch.empty((mr, wl.I * (1 if fp8a else 2)), dtype=torch.uint8, device="cuda")
+    y = torch.empty((mr, wl.H), dtype=torch.float32, device="cuda")
+    out = torch.empty((wl.T, wl.H), dtype=torch.bfloat16, device="cuda")
+    ws = moe.workspace(s)
+    moe.reset_device_status(ws)
+    moe.route_topk(s, L.logits, ids, w)
+    moe.align_permute(s, ids, counts, offsets, rows, inv, ws)
+    moe.gather(s, L.x, rows, offsets, L.a1, xp)
+    moe.grouped_gemm_swiglu(s, xp, L.w13, L.s13, L.a1, a2, offsets, h, ws)
+    moe.grouped_gemm_down(s, h, L.w2, L.s2, a2, offsets, y, ws)
+    moe.combine(s, y, w, inv, offsets, out)
+    torch.cuda.synchronize()
+    assert moe.device_status(ws) == 0
+    return out
+
+
+@pytest.mark.parametrize("wl,variant", STEPWISE, ids=lambda v: getattr(v, "name", str(v)))
+def test_fused_gather_and_combine_equal_the_separate_steps_bit_for_bit(wl, variant):
+    d = syn.make_inputs(wl)
+    a2 = 1.0
+    if wl.adtype == syn.E4M3:
+        a2 = float(np.float32(orc.hidden_amax(d["x"], d["logits"], d["w13"], E=wl.E, k=wl.k, wdtype=syn.E4M3,
+                                              adtype=syn.E4M3, w13_scale=d["w13_scale"], a1=d["a1"],
+                                              tokens=np.arange(16, dtype=np.int32)) / 448))
+    L = Layer(wl, d, variant=variant, a2=a2)
+    L.run()
+    assert L.status() == 0
+    fused = L.out.clone()
+    ref = _stepwise(L, a2)
+    assert torch.equal(fused.view(torch.int16), ref.view(torch.int16))
+    L.run()                                                     # and again: deterministic
+    assert torch.equal(L.out.view(torch.int16), fused.view(torch.int16))
