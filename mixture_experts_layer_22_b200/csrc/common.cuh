@@ -144,6 +144,11 @@ cudaError_t launch_combine(const moe_shape_t &s, const float *y, const float *w,
 // Split bf16 rows [offsets[E+n_shared], K] of `src` into E4M3 planes hi
 // (rows 0..) and lo (rows max_rows..) of `planes` with v = scale[row] *
 // (hi + lo); see small_kernels.cu.
+// Gather + hi/lo split in one pass: the planes of each non-pad slot's token
+// row of x [T, H] (lo plane at row max_rows) and its scale.
+cudaError_t launch_gather_split(const moe_shape_t &s, const void *x, const int32_t *sorted_rows,
+                                const int32_t *offsets, void *planes, float *scale, int64_t max_rows,
+                                cudaStream_t st, bool chained);
 // sorted_rows (may be NULL): skip the rows of pad slots
 cudaError_t launch_split_hilo(const moe_shape_t &s, const void *src, int K, const int32_t *offsets,
                               void *planes, float *scale, int64_t max_rows, cudaStream_t st,
@@ -163,6 +168,11 @@ struct GemmArgs {
     int64_t max_rows;
     bool chained;             // PDL launch; counters already zero
     const int32_t *skip_pad_rows = nullptr;   // the layer's sorted_rows: pad slots' rows need no split
+    bool planes_ready = false;                // hi/lo path, mode 0: the planes of act were made already
+    // Swap-AB mode 0 in the layer: prefetch into L2 this many bytes per CTA of
+    // the down projection's weights (next_wgt) once GEMM1's loads are issued
+    const void *next_wgt = nullptr;
+    long long next_prefetch_bytes = 0;
     void *planes;             // E4M3 weights + bf16 activations: hi/lo activation planes
     float *rowscale;          //   [2 * max_rows, K] E4M3 and the scale of each row
     // fused combine (mode 1): slot -> row code; stage rows in ystage [T, k + n_shared, H],

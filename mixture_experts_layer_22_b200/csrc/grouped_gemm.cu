@@ -79,6 +79,11 @@ struct GemmParams {
     int n_ct;                     // output-feature tiles per token row
     const float *wts;             // router weights [T, k]
     __nv_bfloat16 *comb_out;      // out [T, H]
+    // Swap-AB GEMM1 of the layer: once its own loads are issued, the producer
+    // prefetches into L2 up to next_prefetch_bytes of the down projection's
+    // weights (map tm_next) for the tiles GEMM2 will give this unit first
+    long long next_prefetch_bytes;
+    int next_K, next_n_feat;
 };
 
 template <int kMode, bool kSwap, bool kFp8, int kBN, bool kHiLo = false, bool kPair = false>
@@ -261,7 +266,8 @@ __device__ __forceinline__ void drain_ring(uint64_t *full, int nstages, int stag
 template <int kMode, bool kSwap, bool kFp8, int kBN, bool kHiLo = false, bool kPair = false>
 __global__ void __launch_bounds__(Cfg<kMode, kSwap, kFp8, kBN, kHiLo, kPair>::kThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tm_w,
-                        const __grid_constant__ CUtensorMap tm_x, GemmParams p)
+                        const __grid_constant__ CUtensorMap tm_x,
+                        const __grid_constant__ CUtensorMap tm_next, GemmParams p)
 {
     using C = Cfg<kMode, kSwap, kFp8, kBN, kHiLo, kPair>;
     extern __shared__ uint8_t dyn_smem[];
@@ -498,6 +504,30 @@ __global__ void __launch_bounds__(Cfg<kMode, kSwap, kFp8, kBN, kHiLo, kPair>::kT
                     if (++stage == n_stages) {
                         stage = 0;
                         phase ^= 1u;
+                    }
+                }
+            }
+            if constexpr (kMode == 0 && kSwap) {
+                if (ok && p.next_prefetch_bytes > 0) {
+                    // GEMM2's tile list is GEMM1's with n_ft2 feature tiles of 128
+                    // rows instead of n_ft (the same row tiles per expert)
+                    const int n_ft2 = (p.next_n_feat + 127) / 128;
+                    const int n_tiles2 = s_prefix[Et] / n_ft * n_ft2;
+                    const int KT2 = p.next_K / C::kKStage;
+                    long long budget = p.next_prefetch_bytes;
+                    for (int t = unit; t < n_tiles2 && budget > 0; t += S.G) {
+                        int lo = 0, hi = Et - 1;
+                        while (lo < hi) {
+                            const int mid = (lo + hi + 1) >> 1;
+                            if (s_prefix[mid] / n_ft * n_ft2 <= t) lo = mid;
+                            else hi = mid - 1;
+                        }
+                        const int seg = s_off[lo + 1] - s_off[lo];
+                        const int nrt = (seg + C::kRowsTile - 1) / C::kRowsTile;
+                        const int ft2 = (t - s_prefix[lo] / n_ft * n_ft2) / nrt;
+                        const int wrow = lo * p.next_n_feat + ft2 * 128;
+                        for (int kk = 0; kk < KT2 && budget > 0; ++kk, budget -= 128 * C::kRowBytes)
+                            tma_prefetch_l2_2d(&tm_next, kk * C::kKStage, wrow);
                     }
                 }
             }
@@ -1136,12 +1166,23 @@ static cudaError_t run_gemm(const moe_shape_t &s, const GemmArgs &a, cudaStream_
     // gate/up halves (128) or W2 rows (256); a CTA of a pair: 128
     const uint32_t wbox = kSwap ? (kMode == 0 ? 64 : 128) : (kMode == 0 || kPair ? 128 : 256);
     const uint32_t xbox = kSwap ? 16 : 128;     // Swap-AB loads token rows in 16-row boxes
-    CUtensorMap tm_w, tm_x;
+    CUtensorMap tm_w, tm_x, tm_next;
     static_assert(Cf::kRowBytes == 128, "tensor maps use 128-byte rows with the 128-byte swizzle");
     if (!make_map(&tm_w, a.wgt, u8w, Et * w_rows, K, wbox) ||
         !make_map(&tm_x, a.act, u8, Cf::kPlanes * a.max_rows, K, xbox)) {
         *host_err = MOE_ERR_CUDA;
         return cudaSuccess;
+    }
+    // the down projection's weights [Et * H, I], 128-row boxes, for the L2
+    // prefetch at the end of a Swap-AB GEMM1 (else an unused copy of tm_w)
+    const bool prefetch_next = kMode == 0 && kSwap && a.next_wgt != nullptr;
+    if (prefetch_next) {
+        if (!make_map(&tm_next, a.next_wgt, u8w, static_cast<uint64_t>(Et) * s.H, s.I, 128)) {
+            *host_err = MOE_ERR_CUDA;
+            return cudaSuccess;
+        }
+    } else {
+        tm_next = tm_w;
     }
     GemmParams p;
     p.offsets = a.offsets;
@@ -1170,6 +1211,9 @@ static cudaError_t run_gemm(const moe_shape_t &s, const GemmArgs &a, cudaStream_
     p.n_ct = (s.H + (kSwap ? 127 : 255)) / (kSwap ? 128 : 256);
     p.wts = a.wts;
     p.comb_out = static_cast<__nv_bfloat16 *>(a.comb_out);
+    p.next_prefetch_bytes = prefetch_next ? a.next_prefetch_bytes : 0;
+    p.next_K = s.I;
+    p.next_n_feat = s.H;
     // decode tiles split cheaply (few token columns); prefill tiles carry
     // 128 KB of fp32 partials, so whole tiles are preferred there; CTA pairs
     // take whole tiles only
@@ -1194,9 +1238,10 @@ static cudaError_t run_gemm(const moe_shape_t &s, const GemmArgs &a, cudaStream_
         attr[1].val.programmaticStreamSerializationAllowed = 1;
         cfg.attrs = attr;
         cfg.numAttrs = a.chained ? 2 : 1;
-        return cudaLaunchKernelEx(&cfg, kern, tm_w, tm_x, p);
+        return cudaLaunchKernelEx(&cfg, kern, tm_w, tm_x, tm_next, p);
     } else {
-        return launch_kernel(kern, dim3(sm_count()), dim3(Cf::kThreads), Cf::kDynSmem, st, a.chained, tm_w, tm_x, p);
+        return launch_kernel(kern, dim3(sm_count()), dim3(Cf::kThreads), Cf::kDynSmem, st, a.chained, tm_w, tm_x,
+                             tm_next, p);
     }
 }
 
@@ -1216,13 +1261,15 @@ cudaError_t launch_grouped_gemm(const moe_shape_t &s, const GemmPlan &p, const G
             err = cudaMemsetAsync(a.counters, 0, 2 * kMaxCtas * sizeof(int32_t), st);
             if (err != cudaSuccess) return err;
         }
-        err = launch_split_hilo(s, a.act, a.mode == 0 ? s.H : s.I, a.offsets, a.planes, a.rowscale,
-                                a.max_rows, st, a.chained, a.skip_pad_rows);
-        if (err != cudaSuccess) return err;
-        *launches += 1;
         GemmArgs g = a;
+        if (!(a.mode == 0 && a.planes_ready)) {
+            err = launch_split_hilo(s, a.act, a.mode == 0 ? s.H : s.I, a.offsets, a.planes, a.rowscale,
+                                    a.max_rows, st, a.chained, a.skip_pad_rows);
+            if (err != cudaSuccess) return err;
+            *launches += 1;
+            g.chained = true;      // counters are zero; a dependent launch of the split
+        }
         g.act = a.planes;
-        g.chained = true;          // counters are zero; a dependent launch of the split
 #define MOE_W8(MODE, BN) err = run_gemm<MODE, true, true, BN, true>(s, g, st, host_err)
 #define MOE_W8_BY_BN(MODE)                   \
     switch (p.bn) {                          \

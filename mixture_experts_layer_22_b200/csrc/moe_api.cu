@@ -95,8 +95,10 @@ bool ws_layout(const moe_shape_t &s, WsLayout &L)
     L.inv = o;         o += up256(R * 4);
     L.xp = o;          o += up256(L.max_rows * s.H * ab);
     L.h = o;           o += up256(L.max_rows * s.I * ab);
-    // fused combine: down-projection rows staged per (token, choice) [T, k+S, H] fp32
-    L.y = o;           o += up256(static_cast<size_t>(s.T) * (s.k + s.n_shared) * s.H * 4);
+    // the down projection's rows: in slot order [max_rows, H] fp32 when the
+    // combine is its own pass, or staged per (token, choice) [T, k+S, H] when
+    // it is fused into the GEMM (at most max_rows rows either way)
+    L.y = o;           o += up256(L.max_rows * s.H * 4);
     L.partials = o;    o += up256(static_cast<size_t>(2 * kMaxCtas) * 128 * L.acc_cols * 4);
     // hi/lo E4M3 planes of GEMM1's then GEMM2's activations (reused: the
     // split of h runs after GEMM1 has finished reading the planes of xp)
@@ -353,7 +355,14 @@ static int fused_impl(const moe_shape_t *shape, const void *x, const float *logi
                          reinterpret_cast<int32_t *>(b + L.chunk_base), ctrl, sm, &g_launches, true);
         if (e != cudaSuccess) return MOE_ERR_CUDA;
     }
-    e = launch_gather(s, x, rows, offsets, a1_scale, xp, L.max_rows, sm, true, true);
+    // the gather (E4M3 weights with bf16 activations: gather and hi/lo split
+    // in one pass, straight into the planes GEMM1 reads)
+    const bool w8 = s.wdtype == MOE_E4M3 && s.adtype == MOE_BF16;
+    if (w8)
+        e = launch_gather_split(s, x, rows, offsets, b + L.planes, reinterpret_cast<float *>(b + L.rowscale),
+                                L.max_rows, sm, true);
+    else
+        e = launch_gather(s, x, rows, offsets, a1_scale, xp, L.max_rows, sm, true, true);
     if (e != cudaSuccess) return MOE_ERR_CUDA;
     g_launches += 1;
     const GemmPlan plan = plan_gemm(s);
@@ -370,6 +379,11 @@ static int fused_impl(const moe_shape_t *shape, const void *x, const float *logi
     int host_err = MOE_OK;
     a.mode = 0;
     a.act = xp;
+    a.planes_ready = w8;
+    // decode: GEMM1 prefetches the start of GEMM2's weight stream into L2 as
+    // it finishes, so that the down projection starts on cached weights
+    a.next_wgt = w2;
+    a.next_prefetch_bytes = 512 * 1024;
     a.wgt = w13;
     a.wscale = w13_scale;
     a.ascale = s.adtype == MOE_E4M3 ? a1_scale : 1.0f;
@@ -378,14 +392,22 @@ static int fused_impl(const moe_shape_t *shape, const void *x, const float *logi
     e = launch_grouped_gemm(s, plan, a, sm, &g_launches, &host_err);
     if (host_err != MOE_OK) return host_err;
     if (e != cudaSuccess) return MOE_ERR_CUDA;
-    // GEMM2 with the combine fused into its epilogue: out is written there
+    // GEMM2.  Decode (Swap-AB): the combine is fused into its epilogue, which
+    // writes out; the combine's staging and counting overlap the weight
+    // stream and a launch disappears.  Prefill (CTA pairs): the combine is its
+    // own pass after GEMM2 -- measured faster there, because the epilogue of a
+    // compute-bound 256-row tile has no room for the combine's L2 reads.
+    const bool fuse_combine = plan.swap;
     a.mode = 1;
+    a.planes_ready = false;
+    a.next_wgt = nullptr;
+    a.next_prefetch_bytes = 0;
     a.act = h;
     a.wgt = w2;
     a.wscale = w2_scale;
     a.ascale = s.adtype == MOE_E4M3 ? a2_scale : 1.0f;
     a.out = y;
-    a.combine = true;
+    a.combine = fuse_combine;
     a.sorted_rows = rows;
     a.ystage = y;
     a.tok_cnt = reinterpret_cast<int32_t *>(b + L.tok_cnt);
@@ -395,6 +417,11 @@ static int fused_impl(const moe_shape_t *shape, const void *x, const float *logi
     e = launch_grouped_gemm(s, plan, a, sm, &g_launches, &host_err);
     if (host_err != MOE_OK) return host_err;
     if (e != cudaSuccess) return MOE_ERR_CUDA;
+    if (!fuse_combine) {
+        e = launch_combine(s, y, w, inv, offsets, out, sm, true);
+        if (e != cudaSuccess) return MOE_ERR_CUDA;
+        g_launches += 1;
+    }
     return MOE_OK;
 }
 

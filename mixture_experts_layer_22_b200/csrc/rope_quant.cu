@@ -32,9 +32,13 @@ namespace moe {
 // r / scale, the residual r - q scale is exact in one fused multiply-add, and
 // RN(q + residual rs) is then the correctly rounded quotient (Markstein's
 // theorem on division by reciprocal refinement, "IA-64 and Elementary
-// Functions", 2000).  Quotients here are at most 448 in magnitude and only
-// ones of at least 2^-10 can give a nonzero E4M3 code, far from fp32's
-// overflow and subnormal range where the theorem's hypotheses fail.
+// Functions", 2000).  The residual is a multiple of about 2^(e_r - 46), so it
+// is exact (if need be as a subnormal) for |r| >= 2^-103.  With
+// 2^-60 <= amax <= 2^100 the scale and rs are normal, and an element can only
+// get a nonzero code when |r| >= amax 2^-19 >= 2^-79, well inside that range;
+// smaller elements get a quotient below 2^-10 of the right sign, hence the same
+// code (+-0) as the exact quotient.  For amax outside the range the IEEE
+// division is used.
 __device__ __forceinline__ float div_by_scale(float r, float scale, float rs)
 {
     const float q = __fmul_rn(r, rs);
@@ -63,7 +67,7 @@ __device__ __forceinline__ void load8_bf16(const void *p, float (&y)[8])
 // (interleaved pairs) or the same element of the lane kL/2 ... away
 // (neox pairs, rot_dim a multiple of 16: a shuffle).
 template <int kL, bool kInterleaved>
-__global__ void __launch_bounds__(256) inv_rope_quant_kernel(const __nv_bfloat16 *__restrict__ x,
+__global__ void __launch_bounds__(256, 3) inv_rope_quant_kernel(const __nv_bfloat16 *__restrict__ x,
                                                              const int32_t *__restrict__ positions,
                                                              const float *__restrict__ cos_sin, int T, int n_heads,
                                                              int rot_dim, int max_pos, int hc, uint8_t *q,
@@ -79,8 +83,11 @@ __global__ void __launch_bounds__(256) inv_rope_quant_kernel(const __nv_bfloat16
     const int n_chunks = (n_heads + hc - 1) / hc;
     const long long n_items = static_cast<long long>(T) * n_chunks;
     // this lane's elements j = 8 li + v: rotated or not, first of its pair,
-    // pair index; neox partners sit half / 8 lanes away in the same register
+    // pair index; neox partners sit half / 8 lanes away in the same register.
+    // A lane's 8 elements are all rotated, all passed through, or (a partial
+    // rotary width that is not a multiple of 8) mixed.
     const int pl = half >> 3;
+    const bool all_rot = 8 * li + 8 <= rot_dim, none_rot = 8 * li >= rot_dim;
     bool rotated[8], first[8];
     int pidx[8];
 #pragma unroll
@@ -109,51 +116,76 @@ __global__ void __launch_bounds__(256) inv_rope_quant_kernel(const __nv_bfloat16
             }
             continue;
         }
+        // cos and the sine signed for the element's place in its pair:
+        // a = a' c + b' s, b = b' c + a' (-s), each term rounded, so the same
+        // bits as the difference b' c - a' s
         const float *cs = cos_sin + static_cast<size_t>(p) * rot_dim;
         float c[8], sn[8];
 #pragma unroll
         for (int v = 0; v < 8; ++v) {
             c[v] = rotated[v] ? __ldg(cs + pidx[v]) : 0.0f;
-            sn[v] = rotated[v] ? __ldg(cs + half + pidx[v]) : 0.0f;
+            const float sv = rotated[v] ? __ldg(cs + half + pidx[v]) : 0.0f;
+            sn[v] = first[v] ? sv : -sv;
         }
-        for (int h0 = h_begin; h0 < h_end; h0 += kHpw) {
-            const int h = h0 + sub;
-            const bool live = h < h_end;
-            float y[8];
-            if (live) load8_bf16(x + (row + h) * kHd + 8 * li, y);
-            else
+        // kP passes of kHpw heads at a time: every load of the kP passes is
+        // issued before any is used (more bytes in flight per lane)
+        constexpr int kP = 4;
+        for (int h00 = h_begin; h00 < h_end; h00 += kP * kHpw) {
+            float y[kP][8];
 #pragma unroll
-                for (int v = 0; v < 8; ++v) y[v] = 0.0f;
-            float r[8];
-            float amax = 0.0f;
+            for (int u = 0; u < kP; ++u) {
+                const int h = h00 + u * kHpw + sub;
+                if (h < h_end) load8_bf16(x + (row + h) * kHd + 8 * li, y[u]);
+                else
 #pragma unroll
-            for (int v = 0; v < 8; ++v) {
-                float yp;
-                if (kInterleaved) yp = y[v ^ 1];
-                else yp = __shfl_xor_sync(0xffffffffu, y[v], pl);
-                float val = y[v];
-                if (rotated[v]) {
-                    const float a = __fmul_rn(y[v], c[v]);
-                    const float b = __fmul_rn(yp, sn[v]);
-                    val = first[v] ? __fadd_rn(a, b) : __fsub_rn(a, b);
+                    for (int v = 0; v < 8; ++v) y[u][v] = 0.0f;
+            }
+#pragma unroll
+            for (int u = 0; u < kP; ++u) {
+                const int h = h00 + u * kHpw + sub;
+                if (h00 + u * kHpw >= h_end) break;        // uniform across the warp
+                float yp[8], r[8];
+#pragma unroll
+                for (int v = 0; v < 8; ++v)
+                    yp[v] = kInterleaved ? y[u][v ^ 1] : __shfl_xor_sync(0xffffffffu, y[u][v], pl);
+                if (all_rot) {
+#pragma unroll
+                    for (int v = 0; v < 8; ++v) r[v] = __fadd_rn(__fmul_rn(y[u][v], c[v]), __fmul_rn(yp[v], sn[v]));
+                } else if (none_rot) {
+#pragma unroll
+                    for (int v = 0; v < 8; ++v) r[v] = y[u][v];
+                } else {
+#pragma unroll
+                    for (int v = 0; v < 8; ++v)
+                        r[v] = rotated[v] ? __fadd_rn(__fmul_rn(y[u][v], c[v]), __fmul_rn(yp[v], sn[v])) : y[u][v];
                 }
-                r[v] = val;
-                amax = fmaxf(amax, fabsf(val));
-            }
+                float amax = 0.0f;
 #pragma unroll
-            for (int o = kL / 2; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-            const float sc = amax > 0.0f ? __fdiv_rn(amax, 448.0f) : 1.0f;
-            const float rs = __frcp_rn(sc);
-            uint32_t w[2] = {0u, 0u};
+                for (int v = 0; v < 8; ++v) amax = fmaxf(amax, fabsf(r[v]));
 #pragma unroll
-            for (int v = 0; v < 8; v += 2) {
-                const float2 qq = make_float2(div_by_scale(r[v], sc, rs), div_by_scale(r[v + 1], sc, rs));
-                const uint32_t pair = static_cast<uint32_t>(__nv_cvt_float2_to_fp8x2(qq, __NV_SATFINITE, __NV_E4M3)) & 0xFFFFu;
-                w[v >> 2] |= pair << ((v & 2) * 8);
-            }
-            if (live) {
-                *reinterpret_cast<uint2 *>(q + (row + h) * kHd + 8 * li) = make_uint2(w[0], w[1]);
-                if (li == 0) scales[row + h] = sc;
+                for (int o = kL / 2; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+                const float sc = amax > 0.0f ? __fdiv_rn(amax, 448.0f) : 1.0f;
+                const float rs = __frcp_rn(sc);
+                float qv[8];
+                if (amax >= 0x1p-60f && amax <= 0x1p100f) {
+#pragma unroll
+                    for (int v = 0; v < 8; ++v) qv[v] = div_by_scale(r[v], sc, rs);
+                } else {
+#pragma unroll
+                    for (int v = 0; v < 8; ++v) qv[v] = __fdiv_rn(r[v], sc);
+                }
+                uint32_t w[2] = {0u, 0u};
+#pragma unroll
+                for (int v = 0; v < 8; v += 2) {
+                    const float2 qq = make_float2(qv[v], qv[v + 1]);
+                    const uint32_t pair =
+                        static_cast<uint32_t>(__nv_cvt_float2_to_fp8x2(qq, __NV_SATFINITE, __NV_E4M3)) & 0xFFFFu;
+                    w[v >> 2] |= pair << ((v & 2) * 8);
+                }
+                if (h < h_end) {
+                    *reinterpret_cast<uint2 *>(q + (row + h) * kHd + 8 * li) = make_uint2(w[0], w[1]);
+                    if (li == 0) scales[row + h] = sc;
+                }
             }
         }
     }

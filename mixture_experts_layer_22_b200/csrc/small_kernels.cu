@@ -696,6 +696,62 @@ __global__ void __launch_bounds__(256) split_hilo_kernel(const uint4 *__restrict
     }
 }
 
+// The gather and the hi/lo split in one pass (the fused layer with E4M3
+// weights and bf16 activations): block per slot, the slot's token row read
+// from x, its planes and scale written as split_hilo_kernel writes them.  Pad
+// slots are skipped (their rows reach no real output).
+__global__ void __launch_bounds__(256) gather_split_kernel(const uint4 *__restrict__ x,
+                                                           const int32_t *__restrict__ sorted_rows,
+                                                           const int32_t *__restrict__ offsets, int Et, int T,
+                                                           int k, int H, int64_t lo_rows, uint2 *planes,
+                                                           float *scale)
+{
+    grid_dep_wait();
+    grid_dep_launch();
+    __shared__ float s_red[8];
+    const int total = offsets[Et];
+    const int nv = H / 8;
+    const int R = T * k;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    for (int row = blockIdx.x; row < total; row += gridDim.x) {
+        const int f = sorted_rows[row];
+        if (f < 0) continue;                                    // the same for the whole block
+        const int t = f < R ? f / k : (f - R) % T;
+        const uint4 *r = x + static_cast<size_t>(t) * nv;
+        float m = 0.0f;
+        for (int v = threadIdx.x; v < nv; v += blockDim.x) m = fmaxf(m, abs_max8(__ldg(r + v)));
+        m = warp_max(m);
+        if (lane == 0) s_red[warp] = m;
+        __syncthreads();
+        m = s_red[0];
+#pragma unroll
+        for (int i = 1; i < 8; ++i) m = fmaxf(m, s_red[i]);
+        __syncthreads();                                  // s_red is rewritten by the next row
+        const int e = row_scale_exp(m);
+        const float inv_s = __uint_as_float(static_cast<uint32_t>(127 - e) << 23);   // 2^-e
+        uint2 *ph = planes + static_cast<size_t>(row) * nv;
+        uint2 *pl = planes + static_cast<size_t>(lo_rows + row) * nv;
+        for (int v = threadIdx.x; v < nv; v += blockDim.x) {
+            uint2 hi, lo;
+            split8(__ldg(r + v), inv_s, hi, lo);
+            ph[v] = hi;
+            pl[v] = lo;
+        }
+        if (threadIdx.x == 0) scale[row] = __uint_as_float(static_cast<uint32_t>(127 + e) << 23);
+    }
+}
+
+cudaError_t launch_gather_split(const moe_shape_t &s, const void *x, const int32_t *sorted_rows,
+                                const int32_t *offsets, void *planes, float *scale, int64_t max_rows,
+                                cudaStream_t st, bool chained)
+{
+    int blocks = static_cast<int>(max_rows < 148 * 8 ? max_rows : 148 * 8);
+    if (blocks < 1) blocks = 1;
+    return launch_kernel(gather_split_kernel, dim3(blocks), dim3(256), 0, st, chained, static_cast<const uint4 *>(x),
+                         sorted_rows, offsets, s.E + s.n_shared, s.T, s.k, s.H, max_rows,
+                         static_cast<uint2 *>(planes), scale);
+}
+
 cudaError_t launch_split_hilo(const moe_shape_t &s, const void *src, int K, const int32_t *offsets,
                               void *planes, float *scale, int64_t max_rows, cudaStream_t st, bool chained,
                               const int32_t *sorted_rows)
