@@ -699,6 +699,28 @@ def measure_rope(rw, dev, args, flush):
             "l2": "flushed between timed steps", "launches_per_step": 1}
 
 
+def rope_main(args):
+    """The inverse-rotary + per-head E4M3 step alone (one GPU): a JSON line
+    with its tokens/s and HBM roofline."""
+    import torch
+    rw = syn.ROPE_WORKLOADS[args.workload]
+    if args.T is not None:
+        rw = rw.with_T(args.T)
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    flush = torch.empty(64 * 2 ** 20, dtype=torch.float32, device=dev)
+    r = measure_rope(rw, dev, args, flush)
+    line = {"metric": "inverse-RoPE + per-head E4M3 tokens/s", "value": r["tokens_per_s"], "unit": UNIT,
+            "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": r["ms_per_step"],
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16-in e4m3-out",
+            "data": "synthetic", "config": {"workload": f"{rw.name}: T={rw.T} heads={rw.n_heads} head_dim={rw.head_dim} "
+                                                        f"rot_dim={rw.rot_dim} {'interleaved' if rw.interleaved else 'neox'}",
+                                            "l2": r["l2"]},
+            "roofline": r["roofline"], "gpu_launches": args.steps}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def sweep(args, dev, d_head, weights_head, wl_head):
     """Every configuration besides the headline, measured the same way."""
     import torch
@@ -742,7 +764,8 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default=HEADLINE[0], choices=sorted(syn.WORKLOADS))
+    ap.add_argument("--workload", default=HEADLINE[0], choices=sorted(syn.WORKLOADS) + sorted(syn.ROPE_WORKLOADS),
+                    help="a layer workload, or an attention-side rope_* workload (that step alone)")
     ap.add_argument("--T", type=int, default=None)
     ap.add_argument("--E", type=int, default=None, help="override the routed expert count (small profiling cases)")
     ap.add_argument("--ref-budget", type=float, default=15.0, help="seconds of host time per oracle sample")
@@ -751,6 +774,8 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.workload in syn.ROPE_WORKLOADS:
+        return rope_main(args)
     wl = syn.WORKLOADS[args.workload]
     T = args.T if args.T is not None else (HEADLINE[1] if args.workload == HEADLINE[0] else wl.T)
     wl = wl.with_T(T)
