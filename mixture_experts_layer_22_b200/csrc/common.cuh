@@ -68,11 +68,36 @@ __device__ __forceinline__ void set_status(int32_t *status, int32_t code)
 __device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
+// Every kernel of the library prefers the largest shared-memory carveout: the
+// grouped GEMMs need it, and a small kernel that asked for a different split
+// of the SM's L1 and shared memory would make the SM switch configuration
+// between the launches of one layer call.  Set once per kernel and device.
+inline void prefer_max_smem(const void *kern)
+{
+    static std::mutex m;
+    static const void *done_kern[256];
+    static int done_dev[256];
+    static int n_done = 0;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    std::lock_guard<std::mutex> g(m);
+    for (int i = 0; i < n_done; ++i)
+        if (done_kern[i] == kern && done_dev[i] == dev) return;
+    cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
+    cudaGetLastError();                          // a refusal only leaves the default carveout
+    if (n_done < 256) {
+        done_kern[n_done] = kern;
+        done_dev[n_done] = dev;
+        ++n_done;
+    }
+}
+
 // Launch with the programmatic-stream-serialisation attribute when `pdl`.
 template <typename... KArgs, typename... Args>
 cudaError_t launch_kernel(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
                           bool pdl, Args... args)
 {
+    prefer_max_smem(reinterpret_cast<const void *>(kern));
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = grid;
     cfg.blockDim = block;
@@ -173,6 +198,7 @@ struct GemmArgs {
     // the down projection's weights (next_wgt) once GEMM1's loads are issued
     const void *next_wgt = nullptr;
     long long next_prefetch_bytes = 0;
+    bool next_reverse = false;               // GEMM2 walks its tile list backwards (fused combine)
     void *planes;             // E4M3 weights + bf16 activations: hi/lo activation planes
     float *rowscale;          //   [2 * max_rows, K] E4M3 and the scale of each row
     // fused combine (mode 1): slot -> row code; stage rows in ystage [T, k + n_shared, H],

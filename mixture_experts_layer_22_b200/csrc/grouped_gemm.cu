@@ -83,7 +83,7 @@ struct GemmParams {
     // prefetches into L2 up to next_prefetch_bytes of the down projection's
     // weights (map tm_next) for the tiles GEMM2 will give this unit first
     long long next_prefetch_bytes;
-    int next_K, next_n_feat;
+    int next_K, next_n_feat, next_reverse;
 };
 
 template <int kMode, bool kSwap, bool kFp8, int kBN, bool kHiLo = false, bool kPair = false>
@@ -143,6 +143,7 @@ struct Item {
 
 struct Sched {
     int n_tiles, KT, G, dp_tiles, sk_tiles, sk_ctas;
+    int reverse;       // walk the tile list from its end (schedule position t is tile n_tiles-1-t)
     long long sk_total;
 };
 
@@ -205,7 +206,8 @@ __device__ __forceinline__ bool iter_next(ItemIter &I, const Sched &S, const int
         const int t = I.c + I.i_dp * S.G;
         if (t < S.dp_tiles) {
             ++I.i_dp;
-            tile_coords<kRowsTile, 0>(t, s_prefix, s_off, Et, n_ft, out.e, out.ft, out.rt);
+            tile_coords<kRowsTile, 0>(S.reverse ? S.n_tiles - 1 - t : t, s_prefix, s_off, Et, n_ft, out.e, out.ft,
+                                      out.rt);
             out.kb = 0;
             out.ke = S.KT;
             out.partial = 0;
@@ -220,7 +222,8 @@ __device__ __forceinline__ bool iter_next(ItemIter &I, const Sched &S, const int
     const int kb = static_cast<int>(I.it % S.KT);
     const long long left = I.it_end - I.it;
     const int ke = static_cast<int>(left < S.KT - kb ? kb + left : S.KT);
-    tile_coords<kRowsTile, 0>(S.dp_tiles + tl, s_prefix, s_off, Et, n_ft, out.e, out.ft, out.rt);
+    const int tt = S.dp_tiles + tl;
+    tile_coords<kRowsTile, 0>(S.reverse ? S.n_tiles - 1 - tt : tt, s_prefix, s_off, Et, n_ft, out.e, out.ft, out.rt);
     out.kb = kb;
     out.ke = ke;
     out.partial = !(kb == 0 && ke == S.KT);
@@ -383,6 +386,13 @@ __global__ void __launch_bounds__(Cfg<kMode, kSwap, kFp8, kBN, kHiLo, kPair>::kT
 
     Sched S;
     S.n_tiles = s_prefix[Et];
+    // A Swap-AB down projection walks its tile list backwards.  With the combine
+    // fused, the last expert's tiles would otherwise finish nearly every token
+    // (a shared expert, after all the routed ones), piling the finishing work
+    // into the kernel's tail; backwards it is spread over the routed experts'
+    // tiles.  The standalone call walks the same way, so that both split the
+    // same tiles for stream-K and give the same bits.
+    S.reverse = kMode == 1 && kSwap ? 1 : 0;
     S.KT = p.K / C::kKStage;
     S.G = kPair ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
     const int rem = S.n_tiles % S.G;
@@ -515,7 +525,8 @@ __global__ void __launch_bounds__(Cfg<kMode, kSwap, kFp8, kBN, kHiLo, kPair>::kT
                     const int n_tiles2 = s_prefix[Et] / n_ft * n_ft2;
                     const int KT2 = p.next_K / C::kKStage;
                     long long budget = p.next_prefetch_bytes;
-                    for (int t = unit; t < n_tiles2 && budget > 0; t += S.G) {
+                    for (int ts = unit; ts < n_tiles2 && budget > 0; ts += S.G) {
+                        const int t = p.next_reverse ? n_tiles2 - 1 - ts : ts;   // GEMM2's walk order
                         int lo = 0, hi = Et - 1;
                         while (lo < hi) {
                             const int mid = (lo + hi + 1) >> 1;
@@ -1214,6 +1225,7 @@ static cudaError_t run_gemm(const moe_shape_t &s, const GemmArgs &a, cudaStream_
     p.next_prefetch_bytes = prefetch_next ? a.next_prefetch_bytes : 0;
     p.next_K = s.I;
     p.next_n_feat = s.H;
+    p.next_reverse = a.next_reverse ? 1 : 0;
     // decode tiles split cheaply (few token columns); prefill tiles carry
     // 128 KB of fp32 partials, so whole tiles are preferred there; CTA pairs
     // take whole tiles only

@@ -384,6 +384,7 @@ static int fused_impl(const moe_shape_t *shape, const void *x, const float *logi
     // it finishes, so that the down projection starts on cached weights
     a.next_wgt = w2;
     a.next_prefetch_bytes = 512 * 1024;
+    a.next_reverse = plan.swap;            // GEMM2 fuses the combine (below) and then walks backwards
     a.wgt = w13;
     a.wscale = w13_scale;
     a.ascale = s.adtype == MOE_E4M3 ? a1_scale : 1.0f;

@@ -656,6 +656,60 @@ __device__ __forceinline__ int row_scale_exp(float amax)
     return e < -126 ? -126 : e;
 }
 
+// Split one bf16 row of nv 16-byte vectors into its hi/lo planes and scale,
+// the whole block cooperating.  A row of up to kRowRegs vectors per thread
+// (K <= 8192 for 256 threads) is read once and kept in registers; a longer
+// row is read twice (once for the max magnitude, once to split).
+constexpr int kRowRegs = 4;
+__device__ __forceinline__ void split_row(const uint4 *__restrict__ r, int nv, uint2 *ph, uint2 *pl, float *scale_out,
+                                          float *s_red)
+{
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const bool in_regs = nv <= kRowRegs * static_cast<int>(blockDim.x);
+    uint4 d[kRowRegs];
+    float m = 0.0f;
+    if (in_regs) {
+#pragma unroll
+        for (int i = 0; i < kRowRegs; ++i) {
+            const int v = threadIdx.x + i * blockDim.x;
+            if (v < nv) {
+                d[i] = __ldg(r + v);
+                m = fmaxf(m, abs_max8(d[i]));
+            }
+        }
+    } else {
+        for (int v = threadIdx.x; v < nv; v += blockDim.x) m = fmaxf(m, abs_max8(__ldg(r + v)));
+    }
+    m = warp_max(m);
+    if (lane == 0) s_red[warp] = m;
+    __syncthreads();
+    m = s_red[0];
+    for (int i = 1; i < static_cast<int>(blockDim.x >> 5); ++i) m = fmaxf(m, s_red[i]);
+    __syncthreads();                                  // s_red is rewritten by the next row
+    const int e = row_scale_exp(m);
+    const float inv_s = __uint_as_float(static_cast<uint32_t>(127 - e) << 23);   // 2^-e
+    if (in_regs) {
+#pragma unroll
+        for (int i = 0; i < kRowRegs; ++i) {
+            const int v = threadIdx.x + i * blockDim.x;
+            if (v < nv) {
+                uint2 hi, lo;
+                split8(d[i], inv_s, hi, lo);
+                ph[v] = hi;
+                pl[v] = lo;
+            }
+        }
+    } else {
+        for (int v = threadIdx.x; v < nv; v += blockDim.x) {
+            uint2 hi, lo;
+            split8(__ldg(r + v), inv_s, hi, lo);
+            ph[v] = hi;
+            pl[v] = lo;
+        }
+    }
+    if (threadIdx.x == 0) *scale_out = __uint_as_float(static_cast<uint32_t>(127 + e) << 23);
+}
+
 // One block per permuted row (grid-stride over the rows that exist).  With
 // sorted_rows (inside the fused layer) pad slots are skipped: their rows
 // reach no real output.
@@ -669,30 +723,10 @@ __global__ void __launch_bounds__(256) split_hilo_kernel(const uint4 *__restrict
     __shared__ float s_red[8];
     const int total = offsets[Et];
     const int nv = K / 8;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     for (int row = blockIdx.x; row < total; row += gridDim.x) {
         if (sorted_rows && sorted_rows[row] < 0) continue;       // the same for the whole block
-        const uint4 *r = src + static_cast<size_t>(row) * nv;
-        float m = 0.0f;
-        for (int v = threadIdx.x; v < nv; v += blockDim.x) m = fmaxf(m, abs_max8(r[v]));
-        m = warp_max(m);
-        if (lane == 0) s_red[warp] = m;
-        __syncthreads();
-        m = s_red[0];
-#pragma unroll
-        for (int i = 1; i < 8; ++i) m = fmaxf(m, s_red[i]);
-        __syncthreads();                                  // s_red is rewritten by the next row
-        const int e = row_scale_exp(m);
-        const float inv_s = __uint_as_float(static_cast<uint32_t>(127 - e) << 23);   // 2^-e
-        uint2 *ph = planes + static_cast<size_t>(row) * nv;
-        uint2 *pl = planes + static_cast<size_t>(lo_rows + row) * nv;
-        for (int v = threadIdx.x; v < nv; v += blockDim.x) {
-            uint2 hi, lo;
-            split8(r[v], inv_s, hi, lo);
-            ph[v] = hi;
-            pl[v] = lo;
-        }
-        if (threadIdx.x == 0) scale[row] = __uint_as_float(static_cast<uint32_t>(127 + e) << 23);
+        split_row(src + static_cast<size_t>(row) * nv, nv, planes + static_cast<size_t>(row) * nv,
+                  planes + static_cast<size_t>(lo_rows + row) * nv, scale + row, s_red);
     }
 }
 
@@ -712,32 +746,12 @@ __global__ void __launch_bounds__(256) gather_split_kernel(const uint4 *__restri
     const int total = offsets[Et];
     const int nv = H / 8;
     const int R = T * k;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     for (int row = blockIdx.x; row < total; row += gridDim.x) {
         const int f = sorted_rows[row];
         if (f < 0) continue;                                    // the same for the whole block
         const int t = f < R ? f / k : (f - R) % T;
-        const uint4 *r = x + static_cast<size_t>(t) * nv;
-        float m = 0.0f;
-        for (int v = threadIdx.x; v < nv; v += blockDim.x) m = fmaxf(m, abs_max8(__ldg(r + v)));
-        m = warp_max(m);
-        if (lane == 0) s_red[warp] = m;
-        __syncthreads();
-        m = s_red[0];
-#pragma unroll
-        for (int i = 1; i < 8; ++i) m = fmaxf(m, s_red[i]);
-        __syncthreads();                                  // s_red is rewritten by the next row
-        const int e = row_scale_exp(m);
-        const float inv_s = __uint_as_float(static_cast<uint32_t>(127 - e) << 23);   // 2^-e
-        uint2 *ph = planes + static_cast<size_t>(row) * nv;
-        uint2 *pl = planes + static_cast<size_t>(lo_rows + row) * nv;
-        for (int v = threadIdx.x; v < nv; v += blockDim.x) {
-            uint2 hi, lo;
-            split8(__ldg(r + v), inv_s, hi, lo);
-            ph[v] = hi;
-            pl[v] = lo;
-        }
-        if (threadIdx.x == 0) scale[row] = __uint_as_float(static_cast<uint32_t>(127 + e) << 23);
+        split_row(x + static_cast<size_t>(t) * nv, nv, planes + static_cast<size_t>(row) * nv,
+                  planes + static_cast<size_t>(lo_rows + row) * nv, scale + row, s_red);
     }
 }
 
