@@ -16,10 +16,12 @@
 // with every product and sum rounded on its own (no fused multiply-add) and
 // IEEE division, so a code is decided the same way wherever it is computed.
 //
-// Layout: head_dim / 8 lanes per head, 8 consecutive elements per lane (one
-// 16-byte load), several heads per warp; see the kernel.  HBM-bound once the
-// per-element arithmetic is lean: per head 2*head_dim bytes in, head_dim + 4
-// bytes out.
+// Layout: head_dim / 16 lanes per head, 16 elements per lane in two 16-byte
+// loads chosen so that both elements of every rotary pair sit in the lane,
+// several heads per warp; see the kernel.  HBM-bound once the per-element
+// arithmetic is lean: per head 2*head_dim bytes in, head_dim + 4 bytes out.
+#include <atomic>
+
 #include <cuda_bf16.h>
 #include <cuda_fp8.h>
 
@@ -46,34 +48,63 @@ __device__ __forceinline__ float div_by_scale(float r, float scale, float rs)
     return __fmaf_rn(res, rs, q);
 }
 
-// Eight bf16 values (one 16-byte load) to fp32.
-__device__ __forceinline__ void load8_bf16(const void *p, float (&y)[8])
+// amax / 448 correctly rounded, for normal results: 448 = 7 * 64, and a
+// division by 64 is exact, so RN(amax / 448) = RN(amax / 7) * 2^-6; the
+// division by 7 is the same reciprocal refinement with RN(1/7).
+__device__ __forceinline__ float div448(float amax)
 {
-    const uint4 v = __ldg(reinterpret_cast<const uint4 *>(p));
-    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        y[2 * i] = __uint_as_float(w[i] << 16);
-        y[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
-    }
+    constexpr float kRcp7 = 0.142857149f;       // RN(1/7)
+    const float q = __fmul_rn(amax, kRcp7);
+    const float res = __fmaf_rn(-q, 7.0f, amax);
+    return __fmul_rn(__fmaf_rn(res, kRcp7, q), 0x1p-6f);
 }
 
-// Each head is handled by kL = head_dim / 8 lanes, 8 consecutive elements
-// per lane (one 16-byte load), so a warp processes 32 / kL heads at once and
-// shares the per-head reduction and scale arithmetic among them.  A warp
-// takes one token and a chunk of hc of its heads: the token's position and
-// the rotary coefficients of the lane's 8 elements are loaded once for the
-// chunk.  Pair partners: the neighbouring element of the same lane
-// (interleaved pairs) or the same element of the lane kL/2 ... away
-// (neox pairs, rot_dim a multiple of 16: a shuffle).
+// A pair of fp32 lanes: the packed fp32x2 multiply, add and fused
+// multiply-add of sm_100 take one instruction for two elements, each element
+// rounded exactly like the scalar operation.  The compiler, however, fuses a
+// packed product whose only use is a packed sum into one packed fused
+// multiply-add, explicit rounding modes and --fmad=false notwithstanding
+// (measured: a 1-ulp change in about one head in six).  sum2 therefore forms
+// the separately rounded sum p + q as fma(q, one, p) with `one` a run-time
+// 1.0 the compiler cannot see through: q * one is exact, so the result is
+// RN(p + q), and no product is left to fuse into it.
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
+__device__ __forceinline__ float2 sum2(float2 p, float2 q, float2 one) { return __ffma2_rn(q, one, p); }
+
+__device__ __forceinline__ float lo_bf16(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float hi_bf16(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+// Two E4M3 codes (round to nearest even, saturated), a in the low byte.
+__device__ __forceinline__ uint32_t e4m3x2(float a, float b)
+{
+    return static_cast<uint32_t>(__nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3)) & 0xFFFFu;
+}
+
+// Each head is handled by kL = head_dim / 16 lanes with 16 elements per lane,
+// read as two 8-element chunks (two 16-byte loads), so that every rotary pair
+// has both its elements in one lane:
+//   neox pairs (i, i + rot_dim/2): a rotating lane holds the chunk of first
+//     elements at 8 li and the chunk of their partners at rot_dim/2 + 8 li
+//     (rot_dim a multiple of 16); the remaining lanes hold the passed-through
+//     tail, 16 consecutive elements from rot_dim on;
+//   interleaved pairs (2i, 2i + 1): lane li holds elements 16 li .. 16 li + 15,
+//     eight pairs, each pair one bf16x2 word.
+// A lane's eight pairs form four packs of two, (a'_0, a'_1) and (b'_0, b'_1),
+// and the rotation a = a' c + b' s, b = b' c + a' (-s) takes three packed
+// instructions per pack and output half; the quotient by the head's scale
+// another three per pack.  A warp processes 32 / kL heads at once and takes
+// one token and a chunk of hc of its heads per item: the token's position and
+// the lane's rotary coefficients are loaded once for the chunk.
 template <int kL, bool kInterleaved>
-__global__ void __launch_bounds__(256, 3) inv_rope_quant_kernel(const __nv_bfloat16 *__restrict__ x,
+__global__ void __launch_bounds__(256, 2) inv_rope_quant_kernel(const __nv_bfloat16 *__restrict__ x,
                                                              const int32_t *__restrict__ positions,
                                                              const float *__restrict__ cos_sin, int T, int n_heads,
-                                                             int rot_dim, int max_pos, int hc, uint8_t *q,
+                                                             int rot_dim, int max_pos, int hc, float one, uint8_t *q,
                                                              float *scales, int32_t *status)
 {
-    constexpr int kHd = 8 * kL;
+    const float2 ONE = make_float2(one, one);      // 1.0, passed in (see sum2)
+    constexpr int kHd = 16 * kL;
     constexpr int kHpw = 32 / kL;                  // heads per warp pass
     const int lane = threadIdx.x & 31;
     const int warp_g = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
@@ -82,24 +113,24 @@ __global__ void __launch_bounds__(256, 3) inv_rope_quant_kernel(const __nv_bfloa
     const int half = rot_dim >> 1;
     const int n_chunks = (n_heads + hc - 1) / hc;
     const long long n_items = static_cast<long long>(T) * n_chunks;
-    // this lane's elements j = 8 li + v: rotated or not, first of its pair,
-    // pair index; neox partners sit half / 8 lanes away in the same register.
-    // A lane's 8 elements are all rotated, all passed through, or (a partial
-    // rotary width that is not a multiple of 8) mixed.
-    const int pl = half >> 3;
-    const bool all_rot = 8 * li + 8 <= rot_dim, none_rot = 8 * li >= rot_dim;
-    bool rotated[8], first[8];
-    int pidx[8];
-#pragma unroll
-    for (int v = 0; v < 8; ++v) {
-        const int j = 8 * li + v;
-        rotated[v] = j < rot_dim;
-        if (kInterleaved) {
-            first[v] = (v & 1) == 0;
-            pidx[v] = j >> 1;
+    // the lane's two chunks (element offsets in the head), its first pair
+    // index, and how many of its eight pairs rotate (8: all, 0: none)
+    int off0, off1, n_rot;
+    const int pbase = 8 * li;
+    if (kInterleaved) {
+        off0 = 16 * li;
+        off1 = off0 + 8;
+        n_rot = min(8, max(0, half - pbase));
+    } else {
+        const int npl = half >> 3;                 // rotating lanes
+        if (li < npl) {
+            off0 = 8 * li;
+            off1 = half + 8 * li;
+            n_rot = 8;
         } else {
-            first[v] = j < half;
-            pidx[v] = first[v] ? j : j - half;
+            off0 = rot_dim + 16 * (li - npl);
+            off1 = off0 + 8;
+            n_rot = 0;
         }
     }
     for (long long item = warp_g; item < n_items; item += n_warps) {
@@ -112,78 +143,125 @@ __global__ void __launch_bounds__(256, 3) inv_rope_quant_kernel(const __nv_bfloa
             if (lane == 0 && status) set_status(status, MOE_ERR_DEVICE_CHECK);
             for (int h = h_begin + sub; h < h_end; h += kHpw) {
                 if (li == 0) scales[row + h] = 0.0f;
-                *reinterpret_cast<uint2 *>(q + (row + h) * kHd + 8 * li) = make_uint2(0u, 0u);
+                uint8_t *dst = q + (row + h) * kHd;
+                *reinterpret_cast<uint2 *>(dst + off0) = make_uint2(0u, 0u);
+                *reinterpret_cast<uint2 *>(dst + off1) = make_uint2(0u, 0u);
             }
             continue;
         }
-        // cos and the sine signed for the element's place in its pair:
-        // a = a' c + b' s, b = b' c + a' (-s), each term rounded, so the same
-        // bits as the difference b' c - a' s
+        // c, s and -s of the lane's pairs, packed two pairs at a time
         const float *cs = cos_sin + static_cast<size_t>(p) * rot_dim;
-        float c[8], sn[8];
+        float2 C[4], S[4], NS[4];
 #pragma unroll
-        for (int v = 0; v < 8; ++v) {
-            c[v] = rotated[v] ? __ldg(cs + pidx[v]) : 0.0f;
-            const float sv = rotated[v] ? __ldg(cs + half + pidx[v]) : 0.0f;
-            sn[v] = first[v] ? sv : -sv;
+        for (int i = 0; i < 4; ++i) {
+            const int i0 = 2 * i, i1 = 2 * i + 1;
+            const float c0 = i0 < n_rot ? __ldg(cs + pbase + i0) : 0.0f;
+            const float c1 = i1 < n_rot ? __ldg(cs + pbase + i1) : 0.0f;
+            const float s0 = i0 < n_rot ? __ldg(cs + half + pbase + i0) : 0.0f;
+            const float s1 = i1 < n_rot ? __ldg(cs + half + pbase + i1) : 0.0f;
+            C[i] = make_float2(c0, c1);
+            S[i] = make_float2(s0, s1);
+            NS[i] = make_float2(-s0, -s1);
         }
         // kP passes of kHpw heads at a time: every load of the kP passes is
         // issued before any is used (more bytes in flight per lane)
         constexpr int kP = 4;
         for (int h00 = h_begin; h00 < h_end; h00 += kP * kHpw) {
-            float y[kP][8];
+            uint4 w[kP][2];
 #pragma unroll
             for (int u = 0; u < kP; ++u) {
                 const int h = h00 + u * kHpw + sub;
-                if (h < h_end) load8_bf16(x + (row + h) * kHd + 8 * li, y[u]);
-                else
-#pragma unroll
-                    for (int v = 0; v < 8; ++v) y[u][v] = 0.0f;
+                if (h < h_end) {
+                    const __nv_bfloat16 *src = x + (row + h) * kHd;
+                    w[u][0] = __ldg(reinterpret_cast<const uint4 *>(src + off0));
+                    w[u][1] = __ldg(reinterpret_cast<const uint4 *>(src + off1));
+                } else {
+                    w[u][0] = w[u][1] = make_uint4(0u, 0u, 0u, 0u);
+                }
             }
 #pragma unroll
             for (int u = 0; u < kP; ++u) {
                 const int h = h00 + u * kHpw + sub;
                 if (h00 + u * kHpw >= h_end) break;        // uniform across the warp
-                float yp[8], r[8];
+                const uint32_t ww[8] = {w[u][0].x, w[u][0].y, w[u][0].z, w[u][0].w,
+                                        w[u][1].x, w[u][1].y, w[u][1].z, w[u][1].w};
+                // (a'_0, a'_1) and (b'_0, b'_1) of the lane's pairs 2i, 2i + 1
+                float2 A[4], B[4];
 #pragma unroll
-                for (int v = 0; v < 8; ++v)
-                    yp[v] = kInterleaved ? y[u][v ^ 1] : __shfl_xor_sync(0xffffffffu, y[u][v], pl);
-                if (all_rot) {
+                for (int i = 0; i < 4; ++i) {
+                    if (kInterleaved) {
+                        A[i] = make_float2(lo_bf16(ww[2 * i]), lo_bf16(ww[2 * i + 1]));
+                        B[i] = make_float2(hi_bf16(ww[2 * i]), hi_bf16(ww[2 * i + 1]));
+                    } else {
+                        A[i] = make_float2(lo_bf16(ww[i]), hi_bf16(ww[i]));
+                        B[i] = make_float2(lo_bf16(ww[4 + i]), hi_bf16(ww[4 + i]));
+                    }
+                }
+                // a = a' c + b' s, b = b' c + a' (-s), each product and the sum rounded
+                float2 RA[4], RB[4];
 #pragma unroll
-                    for (int v = 0; v < 8; ++v) r[v] = __fadd_rn(__fmul_rn(y[u][v], c[v]), __fmul_rn(yp[v], sn[v]));
-                } else if (none_rot) {
+                for (int i = 0; i < 4; ++i) {
+                    RA[i] = sum2(mul2(A[i], C[i]), mul2(B[i], S[i]), ONE);
+                    RB[i] = sum2(mul2(B[i], C[i]), mul2(A[i], NS[i]), ONE);
+                }
+                if (n_rot < 8) {
 #pragma unroll
-                    for (int v = 0; v < 8; ++v) r[v] = y[u][v];
-                } else {
-#pragma unroll
-                    for (int v = 0; v < 8; ++v)
-                        r[v] = rotated[v] ? __fadd_rn(__fmul_rn(y[u][v], c[v]), __fmul_rn(yp[v], sn[v])) : y[u][v];
+                    for (int i = 0; i < 4; ++i) {
+                        if (2 * i >= n_rot) { RA[i].x = A[i].x; RB[i].x = B[i].x; }
+                        if (2 * i + 1 >= n_rot) { RA[i].y = A[i].y; RB[i].y = B[i].y; }
+                    }
                 }
                 float amax = 0.0f;
 #pragma unroll
-                for (int v = 0; v < 8; ++v) amax = fmaxf(amax, fabsf(r[v]));
+                for (int i = 0; i < 4; ++i) {
+                    amax = fmaxf(amax, fabsf(RA[i].x));
+                    amax = fmaxf(amax, fabsf(RA[i].y));
+                    amax = fmaxf(amax, fabsf(RB[i].x));
+                    amax = fmaxf(amax, fabsf(RB[i].y));
+                }
 #pragma unroll
                 for (int o = kL / 2; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-                const float sc = amax > 0.0f ? __fdiv_rn(amax, 448.0f) : 1.0f;
-                const float rs = __frcp_rn(sc);
-                float qv[8];
-                if (amax >= 0x1p-60f && amax <= 0x1p100f) {
+                const bool fast = amax >= 0x1p-60f && amax <= 0x1p100f;
+                const float sc = fast ? div448(amax) : (amax > 0.0f ? __fdiv_rn(amax, 448.0f) : 1.0f);
+                float2 QA[4], QB[4];
+                if (fast) {
+                    // reciprocal refinement (div_by_scale), two elements per instruction
+                    const float rs = __frcp_rn(sc);
+                    const float2 RS = make_float2(rs, rs), NSC = make_float2(-sc, -sc);
 #pragma unroll
-                    for (int v = 0; v < 8; ++v) qv[v] = div_by_scale(r[v], sc, rs);
+                    for (int i = 0; i < 4; ++i) {
+                        const float2 qa = mul2(RA[i], RS), qb = mul2(RB[i], RS);
+                        QA[i] = fma2(fma2(qa, NSC, RA[i]), RS, qa);
+                        QB[i] = fma2(fma2(qb, NSC, RB[i]), RS, qb);
+                    }
                 } else {
 #pragma unroll
-                    for (int v = 0; v < 8; ++v) qv[v] = __fdiv_rn(r[v], sc);
+                    for (int i = 0; i < 4; ++i) {
+                        QA[i] = make_float2(__fdiv_rn(RA[i].x, sc), __fdiv_rn(RA[i].y, sc));
+                        QB[i] = make_float2(__fdiv_rn(RB[i].x, sc), __fdiv_rn(RB[i].y, sc));
+                    }
                 }
-                uint32_t w[2] = {0u, 0u};
+                // codes in element order: chunk 0 then chunk 1
+                uint32_t c0[2], c1[2];
+                if (kInterleaved) {
+                    // elements 4i .. 4i + 3 are a_2i, b_2i, a_2i+1, b_2i+1
 #pragma unroll
-                for (int v = 0; v < 8; v += 2) {
-                    const float2 qq = make_float2(qv[v], qv[v + 1]);
-                    const uint32_t pair =
-                        static_cast<uint32_t>(__nv_cvt_float2_to_fp8x2(qq, __NV_SATFINITE, __NV_E4M3)) & 0xFFFFu;
-                    w[v >> 2] |= pair << ((v & 2) * 8);
+                    for (int i = 0; i < 4; ++i) {
+                        const uint32_t wd = e4m3x2(QA[i].x, QB[i].x) | (e4m3x2(QA[i].y, QB[i].y) << 16);
+                        if (i < 2) c0[i] = wd;
+                        else c1[i - 2] = wd;
+                    }
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 2; ++i) {
+                        c0[i] = e4m3x2(QA[2 * i].x, QA[2 * i].y) | (e4m3x2(QA[2 * i + 1].x, QA[2 * i + 1].y) << 16);
+                        c1[i] = e4m3x2(QB[2 * i].x, QB[2 * i].y) | (e4m3x2(QB[2 * i + 1].x, QB[2 * i + 1].y) << 16);
+                    }
                 }
                 if (h < h_end) {
-                    *reinterpret_cast<uint2 *>(q + (row + h) * kHd + 8 * li) = make_uint2(w[0], w[1]);
+                    uint8_t *dst = q + (row + h) * kHd;
+                    *reinterpret_cast<uint2 *>(dst + off0) = make_uint2(c0[0], c0[1]);
+                    *reinterpret_cast<uint2 *>(dst + off1) = make_uint2(c1[0], c1[1]);
                     if (li == 0) scales[row + h] = sc;
                 }
             }
@@ -194,6 +272,25 @@ __global__ void __launch_bounds__(256, 3) inv_rope_quant_kernel(const __nv_bfloa
 }  // namespace moe
 
 using namespace moe;
+
+// Blocks of 256 threads of one kernel variant that fit on the whole GPU at
+// once, cached per variant and device.
+template <int kL, bool kInterleaved>
+static int rope_resident_blocks()
+{
+    static std::atomic<int> cache[64];
+    int dev = 0;
+    cudaGetDevice(&dev);
+    int n = (dev >= 0 && dev < 64) ? cache[dev].load(std::memory_order_relaxed) : 0;
+    if (n == 0) {
+        int sms = 0, per_sm = 0;
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, inv_rope_quant_kernel<kL, kInterleaved>, 256, 0);
+        n = (sms > 0 ? sms : 148) * (per_sm > 0 ? per_sm : 1);
+        if (dev >= 0 && dev < 64) cache[dev].store(n, std::memory_order_relaxed);
+    }
+    return n;
+}
 
 extern "C" int moe_inv_rope_quant_per_head(const moe_rope_shape_t *shape, const void *x, const int32_t *positions,
                                            const float *cos_sin, uint8_t *q, float *scales, int32_t *status,
@@ -217,27 +314,32 @@ extern "C" int moe_inv_rope_quant_per_head(const moe_rope_shape_t *shape, const 
     // heads per warp item: all of a token's heads when there are enough tokens
     // to give every SM 32 warps, else fewer so that small batches still spread
     // over the GPU
-    const int hpw = 32 / (s.head_dim / 8);
+    const int L = s.head_dim / 16;
+    const int hpw = 32 / L;
     int hc = s.n_heads;
     while (hc > hpw && static_cast<long long>(s.num_tokens) * ((s.n_heads + hc - 1) / hc) < 148LL * 32)
         hc = ((hc / 2) + hpw - 1) / hpw * hpw;
     const long long items = static_cast<long long>(s.num_tokens) * ((s.n_heads + hc - 1) / hc);
     const long long want = (items + 7) / 8;
-    const int blocks = static_cast<int>(want < 148 * 8 ? want : 148 * 8);
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     const __nv_bfloat16 *xb = static_cast<const __nv_bfloat16 *>(x);
-#define MOE_ROPE(L, IL)                                                                                      \
-    inv_rope_quant_kernel<L, IL><<<blocks, 256, 0, st>>>(xb, positions, cos_sin, s.num_tokens, s.n_heads,    \
-                                                          s.rot_dim, s.max_pos, hc, q, scales, status)
-    const int L = s.head_dim / 8;
+    // one wave of resident blocks, each warp striding over the items
+#define MOE_ROPE(LL, IL)                                                                                     \
+    do {                                                                                                     \
+        const long long cap = static_cast<long long>(rope_resident_blocks<LL, IL>());                      \
+        const int blocks = static_cast<int>(want < cap ? want : cap);                                        \
+        inv_rope_quant_kernel<LL, IL><<<blocks, 256, 0, st>>>(xb, positions, cos_sin, s.num_tokens,          \
+                                                               s.n_heads, s.rot_dim, s.max_pos, hc, 1.0f, q,  \
+                                                               scales, status);                              \
+    } while (0)
     if (s.interleaved) {
-        if (L == 8) MOE_ROPE(8, true);
-        else if (L == 16) MOE_ROPE(16, true);
-        else MOE_ROPE(32, true);
+        if (L == 4) MOE_ROPE(4, true);
+        else if (L == 8) MOE_ROPE(8, true);
+        else MOE_ROPE(16, true);
     } else {
-        if (L == 8) MOE_ROPE(8, false);
-        else if (L == 16) MOE_ROPE(16, false);
-        else MOE_ROPE(32, false);
+        if (L == 4) MOE_ROPE(4, false);
+        else if (L == 8) MOE_ROPE(8, false);
+        else MOE_ROPE(16, false);
     }
 #undef MOE_ROPE
     launches = 1;

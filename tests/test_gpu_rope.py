@@ -49,6 +49,9 @@ SMALL = [
     syn.RopeWorkload("partial", T=50, n_heads=4, head_dim=128, rot_dim=64, seed=4),
     syn.RopeWorkload("partial_il", T=50, n_heads=4, head_dim=256, rot_dim=96, interleaved=True, seed=5),
     syn.RopeWorkload("rot16", T=9, n_heads=2, head_dim=64, rot_dim=16, seed=6),
+    syn.RopeWorkload("partial96", T=21, n_heads=3, head_dim=128, rot_dim=96, seed=12),
+    syn.RopeWorkload("partial48_hd64", T=19, n_heads=9, head_dim=64, rot_dim=48, seed=13),
+    syn.RopeWorkload("partial_il_odd", T=11, n_heads=2, head_dim=64, rot_dim=22, interleaved=True, seed=14),
     syn.RopeWorkload("rot2_il", T=9, n_heads=3, head_dim=128, rot_dim=2, interleaved=True, seed=10),
     syn.RopeWorkload("many_heads", T=3, n_heads=77, head_dim=64, rot_dim=64, seed=11),
 ]
