@@ -59,12 +59,13 @@ struct GemmParams {
     int lo_rows;             // kHiLo: row offset of the lo plane in the activation map
     int pdl;          // launched as a programmatic dependent: prefetch the first weight
                       // stages into L2 before waiting for the previous kernel
-    int stream_k;     // 0: whole tiles only.  Otherwise whole tiles for all but the
-                      // last one or two rounds, which are split into equal K-step ranges
-                      // (stream-K, each tile shared by at most ~2 CTAs), except that whole
-                      // tiles are used throughout when the rounds are full enough:
-                      // 1 (HBM-bound decode): >= 97% full on average;
-                      // 2 (tensor-bound prefill): >= 90% full on average.
+    int stream_k;     // 0: whole tiles only.  Otherwise the largest idle share, in
+                      // percent of all rounds, that whole tiles may leave: above it the
+                      // tiles of the last one or two rounds are split into equal K-step
+                      // ranges (stream-K, each tile shared by at most ~2 CTAs).
+    int split_cost;   // ... unless the idle whole-tile work per CTA is at most this
+                      // many K-steps: the cost of splitting (a split item's epilogue,
+                      // partial store and fixup) in main-loop K-steps
     const int32_t *sorted_rows;   // slot -> row code (combine)
     int T, k, R, n_shared;        // tokens, top-k, routed rows T*k, shared experts
     // Fused combine (mode 1): instead of y in slot order, each row is staged
@@ -158,19 +159,21 @@ __device__ __forceinline__ long long sk_begin(int c, const Sched &S)
     return static_cast<long long>(c) * S.sk_total / S.sk_ctas;
 }
 
-// Iterator over the work items of CTA `c`: whole tiles c, c+G, ... below
-// dp_tiles, then its contiguous K-step range of the stream-K region.
+// Iterator over the work items of CTA `c`: first its contiguous K-step range
+// of the stream-K region, then whole tiles c, c+G, ... below dp_tiles.  With
+// the split items first, the fixup of a split tile (by its last contributor)
+// overlaps whole-tile main loops instead of landing in the kernel's tail.
 struct ItemIter {
     int c, i_dp;
     long long it, it_end;
-    bool in_sk, first_sk;
+    bool in_dp, first_sk;
 };
 
 __device__ __forceinline__ void iter_init(ItemIter &I, const Sched &S, int c)
 {
     I.c = c;
     I.i_dp = 0;
-    I.in_sk = false;
+    I.in_dp = false;
     I.first_sk = true;
     if (c < S.sk_ctas) {
         I.it = sk_begin(c, S);
@@ -202,35 +205,35 @@ template <int kRowsTile>
 __device__ __forceinline__ bool iter_next(ItemIter &I, const Sched &S, const int *s_prefix,
                                           const int *s_off, int Et, int n_ft, Item &out)
 {
-    if (!I.in_sk) {
-        const int t = I.c + I.i_dp * S.G;
-        if (t < S.dp_tiles) {
-            ++I.i_dp;
-            tile_coords<kRowsTile, 0>(S.reverse ? S.n_tiles - 1 - t : t, s_prefix, s_off, Et, n_ft, out.e, out.ft,
-                                      out.rt);
-            out.kb = 0;
-            out.ke = S.KT;
-            out.partial = 0;
-            out.sk_tile = -1;
-            out.slot = -1;
+    if (!I.in_dp) {
+        if (I.it < I.it_end) {
+            const int tl = static_cast<int>(I.it / S.KT);
+            const int kb = static_cast<int>(I.it % S.KT);
+            const long long left = I.it_end - I.it;
+            const int ke = static_cast<int>(left < S.KT - kb ? kb + left : S.KT);
+            const int tt = S.dp_tiles + tl;
+            tile_coords<kRowsTile, 0>(S.reverse ? S.n_tiles - 1 - tt : tt, s_prefix, s_off, Et, n_ft, out.e,
+                                      out.ft, out.rt);
+            out.kb = kb;
+            out.ke = ke;
+            out.partial = !(kb == 0 && ke == S.KT);
+            out.sk_tile = tl;
+            out.slot = 2 * I.c + (I.first_sk ? 0 : 1);
+            I.first_sk = false;
+            I.it += ke - kb;
             return true;
         }
-        I.in_sk = true;
+        I.in_dp = true;
     }
-    if (I.it >= I.it_end) return false;
-    const int tl = static_cast<int>(I.it / S.KT);
-    const int kb = static_cast<int>(I.it % S.KT);
-    const long long left = I.it_end - I.it;
-    const int ke = static_cast<int>(left < S.KT - kb ? kb + left : S.KT);
-    const int tt = S.dp_tiles + tl;
-    tile_coords<kRowsTile, 0>(S.reverse ? S.n_tiles - 1 - tt : tt, s_prefix, s_off, Et, n_ft, out.e, out.ft, out.rt);
-    out.kb = kb;
-    out.ke = ke;
-    out.partial = !(kb == 0 && ke == S.KT);
-    out.sk_tile = tl;
-    out.slot = 2 * I.c + (I.first_sk ? 0 : 1);
-    I.first_sk = false;
-    I.it += ke - kb;
+    const int t = I.c + I.i_dp * S.G;
+    if (t >= S.dp_tiles) return false;
+    ++I.i_dp;
+    tile_coords<kRowsTile, 0>(S.reverse ? S.n_tiles - 1 - t : t, s_prefix, s_off, Et, n_ft, out.e, out.ft, out.rt);
+    out.kb = 0;
+    out.ke = S.KT;
+    out.partial = 0;
+    out.sk_tile = -1;
+    out.slot = -1;
     return true;
 }
 
@@ -397,13 +400,12 @@ __global__ void __launch_bounds__(Cfg<kMode, kSwap, kFp8, kBN, kHiLo, kPair>::kT
     S.G = kPair ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
     const int rem = S.n_tiles % S.G;
     // whole tiles throughout when the idle share of the last round, over
-    // all rounds, is small: 3% for decode (each SM streams at a bounded
-    // rate, so idle SMs cost time) and 10% for prefill (split tiles carry
-    // 128 KB partials)
+    // all rounds, is at most p.stream_k percent, or when the idle K-steps
+    // per CTA are fewer than a split would cost
     const int rounds = (S.n_tiles + S.G - 1) / S.G;
     const long long idle = static_cast<long long>(S.G) * rounds - S.n_tiles;
-    const bool full_enough = S.n_tiles >= S.G &&
-                             100 * idle <= (p.stream_k == 1 ? 3LL : 10LL) * S.G * rounds;
+    const bool full_enough = S.n_tiles >= S.G && (100 * idle <= static_cast<long long>(p.stream_k) * S.G * rounds ||
+                                                  idle * S.KT <= static_cast<long long>(p.split_cost) * S.G);
     if (!p.stream_k || rem == 0) S.dp_tiles = S.n_tiles;
     else if (S.n_tiles < S.G) S.dp_tiles = 0;
     else if (full_enough) S.dp_tiles = S.n_tiles;
@@ -1195,7 +1197,7 @@ static cudaError_t run_gemm(const moe_shape_t &s, const GemmArgs &a, cudaStream_
     } else {
         tm_next = tm_w;
     }
-    GemmParams p;
+    GemmParams p{};
     p.offsets = a.offsets;
     p.E_tot = Et;
     p.K = K;
@@ -1226,10 +1228,16 @@ static cudaError_t run_gemm(const moe_shape_t &s, const GemmArgs &a, cudaStream_
     p.next_K = s.I;
     p.next_n_feat = s.H;
     p.next_reverse = a.next_reverse ? 1 : 0;
-    // decode tiles split cheaply (few token columns); prefill tiles carry
-    // 128 KB of fp32 partials, so whole tiles are preferred there; CTA pairs
-    // take whole tiles only
-    p.stream_k = kSwap ? 1 : (kPair ? 0 : 2);
+    // When to split tiles.  Decode (Swap-AB): above 3% idle, unless the idle
+    // work is under 12 K-steps per CTA.  A split item's epilogue (partial
+    // store, fixup, combine) costs about that much of the weight stream: on
+    // the DeepSeek-V3 down projection for one token (504 tiles of 16 K-steps
+    // on 148 SMs, 15% idle) whole tiles measured 7% faster than splitting,
+    // while long-K tiles (Mixtral, 224 K-steps) gain from splitting.  Prefill
+    // tiles carry 128 KB of fp32 partials: above 10% idle.  CTA pairs take
+    // whole tiles only.
+    p.stream_k = kSwap ? 3 : (kPair ? 0 : 10);
+    p.split_cost = kSwap ? 12 : 0;
     p.pdl = a.chained ? 1 : 0;
     if (!a.chained) {
         cudaError_t err = cudaMemsetAsync(a.counters, 0, 2 * kMaxCtas * sizeof(int32_t), st);
