@@ -209,32 +209,34 @@ def measured_peaks():
         return 6650.0, 1590.0, 1400.0, "fallback"
 
 
-KERNEL_SOURCES = ("grouped_gemm.cu", "ptx.cuh", "common.cuh")
-
-
-def kernel_source_sha256() -> str:
-    """sha256 over the grouped GEMM's source files, concatenated in order."""
+def source_sha256(names) -> str:
+    """sha256 over the named kernel source files, concatenated in order."""
     import hashlib
     h = hashlib.sha256()
-    for name in KERNEL_SOURCES:
+    for name in names:
         with open(os.path.join(ROOT, "mixture_experts_layer_22_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()
 
 
-def captured_traffic(wl, which: str):
-    """DRAM bytes per launch of a grouped GEMM from the committed ncu capture
-    (profiles/traffic.json), or None when no capture exists for this workload
-    or the kernel source has changed since it was taken."""
+def captured_traffic(key: str):
+    """DRAM bytes per launch of a kernel from a committed ncu capture
+    (profiles/traffic.json, keyed "<workload> T=<T> <kernel>"), or None when
+    no capture exists for it or its kernel sources have changed since."""
     try:
         with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
             t = json.load(f)
-        sha = kernel_source_sha256()
     except (OSError, ValueError):
         return None
-    if sha != t.get("source_sha256"):
-        return None
-    return t.get("kernels", {}).get(f"{wl.name} T={wl.T} {which}")
+    for cap in t.get("captures", []):
+        if key in cap.get("kernels", {}):
+            try:
+                if source_sha256(cap["sources"]) != cap.get("source_sha256"):
+                    return None
+            except OSError:
+                return None
+            return cap["kernels"][key]
+    return None
 
 
 def static_hidden_scale(wl) -> float:
@@ -540,8 +542,8 @@ def measure_workload(wl, d, dev, args, weights=None, full=False, flush=None):
         g["peak_kind"] = peak_kind
     g1["kernel"] = "grouped_gemm gate/up + SwiGLU" + (" (+ hi/lo split)" if (wl.wdtype, wl.adtype) == (1, 0) else "")
     g2["kernel"] = "grouped_gemm down" + (" (+ hi/lo split)" if (wl.wdtype, wl.adtype) == (1, 0) else "")
-    g1["traffic"] = captured_traffic(wl, "gemm1")
-    g2["traffic"] = captured_traffic(wl, "gemm2")
+    g1["traffic"] = captured_traffic(f"{wl.name} T={wl.T} gemm1")
+    g2["traffic"] = captured_traffic(f"{wl.name} T={wl.T} gemm2")
     res["gemm1"], res["gemm2"] = g1, g2
     return res, L
 
@@ -695,7 +697,8 @@ def measure_rope(rw, dev, args, flush):
     return {"T": rw.T, "n_heads": rw.n_heads, "head_dim": rw.head_dim, "rot_dim": rw.rot_dim,
             "interleaved": rw.interleaved, "ms_per_step": ms, "tokens_per_s": rw.T / (ms * 1e-3),
             "roofline": {"bound": "hbm", "achieved": nbytes / (ms * 1e-3) / 1e9, "peak": hbm_peak, "unit": "GB/s",
-                         "frac": nbytes / (ms * 1e-3) / 1e9 / hbm_peak, "algorithmic_bytes": nbytes},
+                         "frac": nbytes / (ms * 1e-3) / 1e9 / hbm_peak, "algorithmic_bytes": nbytes,
+                         "traffic": captured_traffic(f"{rw.name} T={rw.T} rope")},
             "l2": "flushed between timed steps", "launches_per_step": 1}
 
 
