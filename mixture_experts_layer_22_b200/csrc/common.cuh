@@ -209,6 +209,9 @@ struct GemmArgs {
     int32_t *tok_cnt = nullptr;
     const float *wts = nullptr;
     void *comb_out = nullptr;
+    // normal order: which rows of each segment this launch takes (GemmParams)
+    int rsplit = 0;
+    bool wait_at_end = false;
 };
 cudaError_t launch_grouped_gemm(const moe_shape_t &s, const GemmPlan &p, const GemmArgs &a,
                                 cudaStream_t st, int *launches, int *host_err);

@@ -59,6 +59,13 @@ struct GemmParams {
     int lo_rows;             // kHiLo: row offset of the lo plane in the activation map
     int pdl;          // launched as a programmatic dependent: prefetch the first weight
                       // stages into L2 before waiting for the previous kernel
+    int rsplit;       // rows of each expert's segment: 0 all; 1 its whole 256-row
+                      // blocks; 2 the rest (under 256 rows)
+    int wait_at_end;  // the previous kernel is a launch over other rows of the same
+                      // GEMM (the CTA-pair launch before an rsplit = 2 launch):
+                      // nothing read here depends on it, so wait for it only before
+                      // exiting, which keeps dependency waits transitive for the
+                      // kernels after this one
     int stream_k;     // 0: whole tiles only.  Otherwise the largest idle share, in
                       // percent of all rounds, that whole tiles may leave: above it the
                       // tiles of the last one or two rounds are split into equal K-step
@@ -184,7 +191,7 @@ __device__ __forceinline__ void iter_init(ItemIter &I, const Sched &S, int c)
 }
 
 template <int kRowsTile, int kFeatTileUnused>
-__device__ __forceinline__ void tile_coords(int t, const int *s_prefix, const int *s_off, int Et,
+__device__ __forceinline__ void tile_coords(int t, const int *s_prefix, const int *s_lo, const int *s_hi, int Et,
                                             int n_ft, int &e, int &ft, int &rt)
 {
     int lo = 0, hi = Et - 1;                 // largest e with prefix[e] <= t
@@ -194,7 +201,7 @@ __device__ __forceinline__ void tile_coords(int t, const int *s_prefix, const in
         else hi = mid - 1;
     }
     e = lo;
-    const int seg = s_off[e + 1] - s_off[e];
+    const int seg = s_hi[e] - s_lo[e];
     const int nrt = (seg + kRowsTile - 1) / kRowsTile;
     const int local = t - s_prefix[e];
     rt = local % nrt;
@@ -203,7 +210,7 @@ __device__ __forceinline__ void tile_coords(int t, const int *s_prefix, const in
 
 template <int kRowsTile>
 __device__ __forceinline__ bool iter_next(ItemIter &I, const Sched &S, const int *s_prefix,
-                                          const int *s_off, int Et, int n_ft, Item &out)
+                                          const int *s_lo, const int *s_hi, int Et, int n_ft, Item &out)
 {
     if (!I.in_dp) {
         if (I.it < I.it_end) {
@@ -212,7 +219,7 @@ __device__ __forceinline__ bool iter_next(ItemIter &I, const Sched &S, const int
             const long long left = I.it_end - I.it;
             const int ke = static_cast<int>(left < S.KT - kb ? kb + left : S.KT);
             const int tt = S.dp_tiles + tl;
-            tile_coords<kRowsTile, 0>(S.reverse ? S.n_tiles - 1 - tt : tt, s_prefix, s_off, Et, n_ft, out.e,
+            tile_coords<kRowsTile, 0>(S.reverse ? S.n_tiles - 1 - tt : tt, s_prefix, s_lo, s_hi, Et, n_ft, out.e,
                                       out.ft, out.rt);
             out.kb = kb;
             out.ke = ke;
@@ -228,7 +235,8 @@ __device__ __forceinline__ bool iter_next(ItemIter &I, const Sched &S, const int
     const int t = I.c + I.i_dp * S.G;
     if (t >= S.dp_tiles) return false;
     ++I.i_dp;
-    tile_coords<kRowsTile, 0>(S.reverse ? S.n_tiles - 1 - t : t, s_prefix, s_off, Et, n_ft, out.e, out.ft, out.rt);
+    tile_coords<kRowsTile, 0>(S.reverse ? S.n_tiles - 1 - t : t, s_prefix, s_lo, s_hi, Et, n_ft, out.e, out.ft,
+                              out.rt);
     out.kb = 0;
     out.ke = S.KT;
     out.partial = 0;
@@ -277,7 +285,9 @@ __global__ void __launch_bounds__(Cfg<kMode, kSwap, kFp8, kBN, kHiLo, kPair>::kT
 {
     using C = Cfg<kMode, kSwap, kFp8, kBN, kHiLo, kPair>;
     extern __shared__ uint8_t dyn_smem[];
-    __shared__ int s_off[kMaxExpertsTotal + 1];
+    // rows [s_lo[e], s_hi[e]) of expert e's padded segment are this launch's
+    // (all of it, or with p.rsplit its whole 256-row blocks or the rest)
+    __shared__ int s_lo[kMaxExpertsTotal], s_hi[kMaxExpertsTotal];
     __shared__ int s_prefix[kMaxExpertsTotal + 1];
     __shared__ __align__(8) uint64_t s_full[C::kSlots], s_empty[C::kSlots];
     __shared__ int s_max_seg;
@@ -343,16 +353,21 @@ __global__ void __launch_bounds__(Cfg<kMode, kSwap, kFp8, kBN, kHiLo, kPair>::kT
     if (warp == 2) {
         // L2 load: under PDL this runs before grid_dep_wait(); the offsets
         // come from the align kernel, which has completed by then
-        for (int e = lane; e <= Et; e += 32) s_off[e] = __ldcg(p.offsets + e);
+        bool bad = false;
+        for (int e = lane; e < Et; e += 32) {
+            const int a = __ldcg(p.offsets + e), b = __ldcg(p.offsets + e + 1);
+            if (b < a || ((b - a) & 15) != 0 || (a & 15) != 0) bad = true;
+            const int blocks = b > a ? a + (b - a) / 256 * 256 : a;   // end of the whole 256-row blocks
+            s_lo[e] = p.rsplit == 2 ? blocks : a;
+            s_hi[e] = p.rsplit == 1 ? blocks : b;
+        }
         __syncwarp();
         const int per = (Et + 31) / 32;
         const int lo = min(Et, lane * per), hi = min(Et, lo + per);
         int sum = 0, mx = 0;
-        bool bad = false;
         for (int e = lo; e < hi; ++e) {
-            const int seg = s_off[e + 1] - s_off[e];
+            const int seg = s_hi[e] - s_lo[e];
             mx = max(mx, seg);
-            if (seg < 0 || (seg & 15) != 0 || (s_off[e] & 15) != 0) bad = true;
             sum += seg > 0 ? ((seg + C::kRowsTile - 1) / C::kRowsTile) * n_ft : 0;
         }
         int inc = sum;
@@ -364,7 +379,7 @@ __global__ void __launch_bounds__(Cfg<kMode, kSwap, kFp8, kBN, kHiLo, kPair>::kT
         int run = inc - sum;
         for (int e = lo; e < hi; ++e) {
             s_prefix[e] = run;
-            const int seg = s_off[e + 1] - s_off[e];
+            const int seg = s_hi[e] - s_lo[e];
             run += seg > 0 ? ((seg + C::kRowsTile - 1) / C::kRowsTile) * n_ft : 0;
         }
         if (lane == 31) s_prefix[Et] = inc;
@@ -426,7 +441,7 @@ __global__ void __launch_bounds__(Cfg<kMode, kSwap, kFp8, kBN, kHiLo, kPair>::kT
         iter_init(I, S, unit);
         Item it;
         int n = 0;
-        while (n < n_stages && iter_next<C::kRowsTile>(I, S, s_prefix, s_off, Et, n_ft, it)) {
+        while (n < n_stages && iter_next<C::kRowsTile>(I, S, s_prefix, s_lo, s_hi, Et, n_ft, it)) {
             const int wbase = it.e * p.w_rows;
             for (int kk = it.kb; kk < it.ke && n < n_stages; ++kk, ++n) {
                 const int kx = kk * C::kKStage;
@@ -443,7 +458,7 @@ __global__ void __launch_bounds__(Cfg<kMode, kSwap, kFp8, kBN, kHiLo, kPair>::kT
             }
         }
     }
-    grid_dep_wait();
+    if (!p.wait_at_end) grid_dep_wait();
     grid_dep_launch();
 
 
@@ -463,9 +478,9 @@ __global__ void __launch_bounds__(Cfg<kMode, kSwap, kFp8, kBN, kHiLo, kPair>::kT
             iter_init(I, S, unit);
             Item it;
             bool ok = true;
-            while (ok && iter_next<C::kRowsTile>(I, S, s_prefix, s_off, Et, n_ft, it)) {
-                const int row0 = s_off[it.e] + it.rt * C::kRowsTile;
-                const int rows = min(C::kRowsTile, s_off[it.e + 1] - row0);
+            while (ok && iter_next<C::kRowsTile>(I, S, s_prefix, s_lo, s_hi, Et, n_ft, it)) {
+                const int row0 = s_lo[it.e] + it.rt * C::kRowsTile;
+                const int rows = min(C::kRowsTile, s_hi[it.e] - row0);
                 const int wbase = it.e * p.w_rows;
                 for (int kk = it.kb; kk < it.ke; ++kk) {
                     if (!mbar_wait(smem_u32(&s_empty[stage]), phase ^ 1u, &s_abort)) {
@@ -535,7 +550,7 @@ __global__ void __launch_bounds__(Cfg<kMode, kSwap, kFp8, kBN, kHiLo, kPair>::kT
                             if (s_prefix[mid] / n_ft * n_ft2 <= t) lo = mid;
                             else hi = mid - 1;
                         }
-                        const int seg = s_off[lo + 1] - s_off[lo];
+                        const int seg = s_hi[lo] - s_lo[lo];
                         const int nrt = (seg + C::kRowsTile - 1) / C::kRowsTile;
                         const int ft2 = (t - s_prefix[lo] / n_ft * n_ft2) / nrt;
                         const int wrow = lo * p.next_n_feat + ft2 * 128;
@@ -570,13 +585,13 @@ __global__ void __launch_bounds__(Cfg<kMode, kSwap, kFp8, kBN, kHiLo, kPair>::kT
             auto wait_bar = [&](uint32_t bar, uint32_t parity) -> bool {
                 return kPair ? mbar_wait_cluster(bar, parity, &s_abort) : mbar_wait(bar, parity, &s_abort);
             };
-            while (ok && iter_next<C::kRowsTile>(I, S, s_prefix, s_off, Et, n_ft, it)) {
+            while (ok && iter_next<C::kRowsTile>(I, S, s_prefix, s_lo, s_hi, Et, n_ft, it)) {
                 if (!wait_bar(smem_u32(&s_tempty[acc]), acc_phase ^ 1u)) break;
                 tc_fence_after();
                 const uint32_t d = tmem_base + acc * C::kAccCols;
                 int n = 256;
                 if (kSwap) {
-                    const int seg = s_off[it.e + 1] - s_off[it.e];
+                    const int seg = s_hi[it.e] - s_lo[it.e];
                     n = C::kPlanes * min(C::kRowsTile, seg - it.rt * C::kRowsTile);
                 }
                 const uint32_t idesc = idesc_make(C::kFmt, kPair ? 256 : 128, n);
@@ -635,14 +650,14 @@ __global__ void __launch_bounds__(Cfg<kMode, kSwap, kFp8, kBN, kHiLo, kPair>::kT
         ItemIter I;
         iter_init(I, S, unit);
         Item it;
-        while (iter_next<C::kRowsTile>(I, S, s_prefix, s_off, Et, n_ft, it)) {
+        while (iter_next<C::kRowsTile>(I, S, s_prefix, s_lo, s_hi, Et, n_ft, it)) {
             const bool got = kPair ? mbar_wait_cluster(smem_u32(&s_tfull[acc]), acc_phase, &s_abort)
                                    : mbar_wait(smem_u32(&s_tfull[acc]), acc_phase, &s_abort);
             if (!named_bar_and(1, C::kEpiThreads, got)) break;   // all epilogue warps agree
             tc_fence_after();
-            const int seg = s_off[it.e + 1] - s_off[it.e];
+            const int seg = s_hi[it.e] - s_lo[it.e];
             // kPair: this CTA holds rows [128 rank, 128 rank + 128) of the pair's tile
-            const int row0 = s_off[it.e] + it.rt * C::kRowsTile + (kPair ? 128 * static_cast<int>(rank) : 0);
+            const int row0 = s_lo[it.e] + it.rt * C::kRowsTile + (kPair ? 128 * static_cast<int>(rank) : 0);
             const int rows = kPair ? max(0, min(128, seg - it.rt * C::kRowsTile - 128 * static_cast<int>(rank)))
                                    : min(C::kRowsTile, seg - it.rt * C::kRowsTile);
             // output scale of the tile; kHiLo: times the activation row's own
@@ -1047,6 +1062,7 @@ __global__ void __launch_bounds__(Cfg<kMode, kSwap, kFp8, kBN, kHiLo, kPair>::kT
         if constexpr (kPair) tmem_dealloc_pair(tmem_base, C::kTmemCols);
         else tmem_dealloc(tmem_base, C::kTmemCols);
     }
+    if (p.wait_at_end) grid_dep_wait();
 }
 
 // ------------------------------------------------------------------ host side
@@ -1228,15 +1244,18 @@ static cudaError_t run_gemm(const moe_shape_t &s, const GemmArgs &a, cudaStream_
     p.next_K = s.I;
     p.next_n_feat = s.H;
     p.next_reverse = a.next_reverse ? 1 : 0;
+    p.rsplit = a.rsplit;
+    p.wait_at_end = a.wait_at_end ? 1 : 0;
     // When to split tiles.  Decode (Swap-AB): above 3% idle, unless the idle
     // work is under 12 K-steps per CTA.  A split item's epilogue (partial
     // store, fixup, combine) costs about that much of the weight stream: on
     // the DeepSeek-V3 down projection for one token (504 tiles of 16 K-steps
     // on 148 SMs, 15% idle) whole tiles measured 7% faster than splitting,
     // while long-K tiles (Mixtral, 224 K-steps) gain from splitting.  Prefill
-    // tiles carry 128 KB of fp32 partials: above 10% idle.  CTA pairs take
-    // whole tiles only.
-    p.stream_k = kSwap ? 3 : (kPair ? 0 : 10);
+    // (normal order) takes whole tiles: a split tile carries 128 KB of fp32
+    // partials, and splitting the one-CTA launch over the segments' last rows
+    // made the Qwen2 and Mixtral down projections 35-40% slower.
+    p.stream_k = kSwap ? 3 : 0;
     p.split_cost = kSwap ? 12 : 0;
     p.pdl = a.chained ? 1 : 0;
     if (!a.chained) {
@@ -1319,16 +1338,33 @@ cudaError_t launch_grouped_gemm(const moe_shape_t &s, const GemmPlan &p, const G
             if (fp8) { MOE_BY_BN(1, true) } else { MOE_BY_BN(1, false) }
         }
     } else {
-        // Normal order.  The down projection runs on CTA pairs (256 x 256
-        // tiles, half the weight bytes staged per SM); the gate/up GEMM keeps
-        // one-CTA 128-row tiles: with many small experts the pairs' 256-row
-        // tiles pad more rows than their operand savings gain back (measured).
+        // Normal order (prefill).  Each expert's whole 256-row blocks run on
+        // CTA pairs (256 x 256 tiles, half the weight bytes staged per SM),
+        // then the rest of its segment (under 256 rows) on one-CTA 128-row
+        // tiles, which pad at most 127 rows per expert where a pair tile pads
+        // up to 255.  The second launch reads nothing the first writes: it
+        // starts as the pairs' SMs free up and waits for them only before
+        // exiting.
+        GemmArgs g = a;
+        g.rsplit = 1;
         if (a.mode == 0) {
-            if (fp8) MOE_G(0, false, true, 256);
-            else MOE_G(0, false, false, 256);
+            if (fp8) err = run_gemm<0, false, true, 128, false, true>(s, g, st, host_err);
+            else err = run_gemm<0, false, false, 128, false, true>(s, g, st, host_err);
         } else {
-            if (fp8) err = run_gemm<1, false, true, 128, false, true>(s, a, st, host_err);
-            else err = run_gemm<1, false, false, 128, false, true>(s, a, st, host_err);
+            if (fp8) err = run_gemm<1, false, true, 128, false, true>(s, g, st, host_err);
+            else err = run_gemm<1, false, false, 128, false, true>(s, g, st, host_err);
+        }
+        if (err != cudaSuccess || *host_err != MOE_OK) return err;
+        *launches += 1;
+        g.rsplit = 2;
+        g.chained = true;
+        g.wait_at_end = true;
+        if (a.mode == 0) {
+            if (fp8) err = run_gemm<0, false, true, 256>(s, g, st, host_err);
+            else err = run_gemm<0, false, false, 256>(s, g, st, host_err);
+        } else {
+            if (fp8) err = run_gemm<1, false, true, 256>(s, g, st, host_err);
+            else err = run_gemm<1, false, false, 256>(s, g, st, host_err);
         }
     }
 #undef MOE_BY_BN

@@ -38,14 +38,14 @@ namespace moe {
 // is exact (if need be as a subnormal) for |r| >= 2^-103.  With
 // 2^-60 <= amax <= 2^100 the scale and rs are normal, and an element can only
 // get a nonzero code when |r| >= amax 2^-19 >= 2^-79, well inside that range;
-// smaller elements get a quotient below 2^-10 of the right sign, hence the same
-// code (+-0) as the exact quotient.  For amax outside the range the IEEE
-// division is used.
-__device__ __forceinline__ float div_by_scale(float r, float scale, float rs)
+// smaller elements get a quotient below 2^-10, hence the code +-0 of the
+// exact quotient, once the sign is right.  The sign needs one fix: for
+// r = -0, q is -0 and the residual +0, and their sum rounds to +0.  The
+// quotient of r by a positive scale has r's sign, so it is taken from r
+// (with_sign_of).  For amax outside the range the IEEE division is used.
+__device__ __forceinline__ float with_sign_of(float q, float r)
 {
-    const float q = __fmul_rn(r, rs);
-    const float res = __fmaf_rn(-q, scale, r);
-    return __fmaf_rn(res, rs, q);
+    return __int_as_float((__float_as_int(q) & 0x7FFFFFFF) | (__float_as_int(r) & static_cast<int>(0x80000000u)));
 }
 
 // amax / 448 correctly rounded, for normal results: 448 = 7 * 64, and a
@@ -81,6 +81,139 @@ __device__ __forceinline__ uint32_t e4m3x2(float a, float b)
     return static_cast<uint32_t>(__nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3)) & 0xFFFFu;
 }
 
+// c, s and -s of the lane's pairs pbase .. pbase + 7 (zero past n_rot) from
+// the position's table row, packed two pairs at a time.
+__device__ __forceinline__ void load_coeffs(const float *cs, int pbase, int half, int n_rot, float2 (&C)[4],
+                                            float2 (&S)[4], float2 (&NS)[4])
+{
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int i0 = 2 * i, i1 = 2 * i + 1;
+        const float c0 = i0 < n_rot ? __ldg(cs + pbase + i0) : 0.0f;
+        const float c1 = i1 < n_rot ? __ldg(cs + pbase + i1) : 0.0f;
+        const float s0 = i0 < n_rot ? __ldg(cs + half + pbase + i0) : 0.0f;
+        const float s1 = i1 < n_rot ? __ldg(cs + half + pbase + i1) : 0.0f;
+        C[i] = make_float2(c0, c1);
+        S[i] = make_float2(s0, s1);
+        NS[i] = make_float2(-s0, -s1);
+    }
+}
+
+// The lane's two 8-element chunks (element offsets in the head), its first
+// pair index, and how many of its eight pairs rotate (8: all, 0: none).
+template <int kL, bool kInterleaved>
+__device__ __forceinline__ void lane_layout(int li, int rot_dim, int &off0, int &off1, int &pbase, int &n_rot)
+{
+    const int half = rot_dim >> 1;
+    pbase = 8 * li;
+    if (kInterleaved) {
+        off0 = 16 * li;
+        off1 = off0 + 8;
+        n_rot = min(8, max(0, half - pbase));
+    } else {
+        const int npl = half >> 3;                 // rotating lanes
+        if (li < npl) {
+            off0 = 8 * li;
+            off1 = half + 8 * li;
+            n_rot = 8;
+        } else {
+            off0 = rot_dim + 16 * (li - npl);
+            off1 = off0 + 8;
+            n_rot = 0;
+        }
+    }
+}
+
+// One head's 16 elements in this lane (chunks w0, w1): rotation, the head's
+// scale (a reduction over its kL lanes; every lane of the warp must call this
+// together) and the codes, which are stored when `store`.
+template <int kL, bool kInterleaved>
+__device__ __forceinline__ void rope_head(const uint4 w0, const uint4 w1, const float2 (&C)[4], const float2 (&S)[4],
+                                          const float2 (&NS)[4], float2 ONE, int n_rot, bool store, uint8_t *dst,
+                                          int off0, int off1, float *scale_dst, int li)
+{
+    const uint32_t ww[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+    // (a'_0, a'_1) and (b'_0, b'_1) of the lane's pairs 2i, 2i + 1
+    float2 A[4], B[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        if (kInterleaved) {
+            A[i] = make_float2(lo_bf16(ww[2 * i]), lo_bf16(ww[2 * i + 1]));
+            B[i] = make_float2(hi_bf16(ww[2 * i]), hi_bf16(ww[2 * i + 1]));
+        } else {
+            A[i] = make_float2(lo_bf16(ww[i]), hi_bf16(ww[i]));
+            B[i] = make_float2(lo_bf16(ww[4 + i]), hi_bf16(ww[4 + i]));
+        }
+    }
+    // a = a' c + b' s, b = b' c + a' (-s), each product and the sum rounded
+    float2 RA[4], RB[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        RA[i] = sum2(mul2(A[i], C[i]), mul2(B[i], S[i]), ONE);
+        RB[i] = sum2(mul2(B[i], C[i]), mul2(A[i], NS[i]), ONE);
+    }
+    if (n_rot < 8) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            if (2 * i >= n_rot) { RA[i].x = A[i].x; RB[i].x = B[i].x; }
+            if (2 * i + 1 >= n_rot) { RA[i].y = A[i].y; RB[i].y = B[i].y; }
+        }
+    }
+    float amax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        amax = fmaxf(amax, fabsf(RA[i].x));
+        amax = fmaxf(amax, fabsf(RA[i].y));
+        amax = fmaxf(amax, fabsf(RB[i].x));
+        amax = fmaxf(amax, fabsf(RB[i].y));
+    }
+#pragma unroll
+    for (int o = kL / 2; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    const bool fast = amax >= 0x1p-60f && amax <= 0x1p100f;
+    const float sc = fast ? div448(amax) : (amax > 0.0f ? __fdiv_rn(amax, 448.0f) : 1.0f);
+    float2 QA[4], QB[4];
+    if (fast) {
+        // reciprocal refinement (see with_sign_of), two elements per instruction
+        const float rs = __frcp_rn(sc);
+        const float2 RS = make_float2(rs, rs), NSC = make_float2(-sc, -sc);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float2 qa = mul2(RA[i], RS), qb = mul2(RB[i], RS);
+            const float2 ta = fma2(fma2(qa, NSC, RA[i]), RS, qa), tb = fma2(fma2(qb, NSC, RB[i]), RS, qb);
+            QA[i] = make_float2(with_sign_of(ta.x, RA[i].x), with_sign_of(ta.y, RA[i].y));
+            QB[i] = make_float2(with_sign_of(tb.x, RB[i].x), with_sign_of(tb.y, RB[i].y));
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            QA[i] = make_float2(__fdiv_rn(RA[i].x, sc), __fdiv_rn(RA[i].y, sc));
+            QB[i] = make_float2(__fdiv_rn(RB[i].x, sc), __fdiv_rn(RB[i].y, sc));
+        }
+    }
+    // codes in element order: chunk 0 then chunk 1
+    uint32_t c0[2], c1[2];
+    if (kInterleaved) {
+        // elements 4i .. 4i + 3 are a_2i, b_2i, a_2i+1, b_2i+1
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const uint32_t wd = e4m3x2(QA[i].x, QB[i].x) | (e4m3x2(QA[i].y, QB[i].y) << 16);
+            if (i < 2) c0[i] = wd;
+            else c1[i - 2] = wd;
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+            c0[i] = e4m3x2(QA[2 * i].x, QA[2 * i].y) | (e4m3x2(QA[2 * i + 1].x, QA[2 * i + 1].y) << 16);
+            c1[i] = e4m3x2(QB[2 * i].x, QB[2 * i].y) | (e4m3x2(QB[2 * i + 1].x, QB[2 * i + 1].y) << 16);
+        }
+    }
+    if (store) {
+        *reinterpret_cast<uint2 *>(dst + off0) = make_uint2(c0[0], c0[1]);
+        *reinterpret_cast<uint2 *>(dst + off1) = make_uint2(c1[0], c1[1]);
+        if (li == 0) *scale_dst = sc;
+    }
+}
+
 // Each head is handled by kL = head_dim / 16 lanes with 16 elements per lane,
 // read as two 8-element chunks (two 16-byte loads), so that every rotary pair
 // has both its elements in one lane:
@@ -113,26 +246,8 @@ __global__ void __launch_bounds__(256, 2) inv_rope_quant_kernel(const __nv_bfloa
     const int half = rot_dim >> 1;
     const int n_chunks = (n_heads + hc - 1) / hc;
     const long long n_items = static_cast<long long>(T) * n_chunks;
-    // the lane's two chunks (element offsets in the head), its first pair
-    // index, and how many of its eight pairs rotate (8: all, 0: none)
-    int off0, off1, n_rot;
-    const int pbase = 8 * li;
-    if (kInterleaved) {
-        off0 = 16 * li;
-        off1 = off0 + 8;
-        n_rot = min(8, max(0, half - pbase));
-    } else {
-        const int npl = half >> 3;                 // rotating lanes
-        if (li < npl) {
-            off0 = 8 * li;
-            off1 = half + 8 * li;
-            n_rot = 8;
-        } else {
-            off0 = rot_dim + 16 * (li - npl);
-            off1 = off0 + 8;
-            n_rot = 0;
-        }
-    }
+    int off0, off1, pbase, n_rot;
+    lane_layout<kL, kInterleaved>(li, rot_dim, off0, off1, pbase, n_rot);
     for (long long item = warp_g; item < n_items; item += n_warps) {
         const int t = static_cast<int>(item / n_chunks);
         const int h_begin = static_cast<int>(item % n_chunks) * hc;
@@ -149,20 +264,8 @@ __global__ void __launch_bounds__(256, 2) inv_rope_quant_kernel(const __nv_bfloa
             }
             continue;
         }
-        // c, s and -s of the lane's pairs, packed two pairs at a time
-        const float *cs = cos_sin + static_cast<size_t>(p) * rot_dim;
         float2 C[4], S[4], NS[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const int i0 = 2 * i, i1 = 2 * i + 1;
-            const float c0 = i0 < n_rot ? __ldg(cs + pbase + i0) : 0.0f;
-            const float c1 = i1 < n_rot ? __ldg(cs + pbase + i1) : 0.0f;
-            const float s0 = i0 < n_rot ? __ldg(cs + half + pbase + i0) : 0.0f;
-            const float s1 = i1 < n_rot ? __ldg(cs + half + pbase + i1) : 0.0f;
-            C[i] = make_float2(c0, c1);
-            S[i] = make_float2(s0, s1);
-            NS[i] = make_float2(-s0, -s1);
-        }
+        load_coeffs(cos_sin + static_cast<size_t>(p) * rot_dim, pbase, half, n_rot, C, S, NS);
         // kP passes of kHpw heads at a time: every load of the kP passes is
         // issued before any is used (more bytes in flight per lane)
         constexpr int kP = 4;
@@ -183,87 +286,8 @@ __global__ void __launch_bounds__(256, 2) inv_rope_quant_kernel(const __nv_bfloa
             for (int u = 0; u < kP; ++u) {
                 const int h = h00 + u * kHpw + sub;
                 if (h00 + u * kHpw >= h_end) break;        // uniform across the warp
-                const uint32_t ww[8] = {w[u][0].x, w[u][0].y, w[u][0].z, w[u][0].w,
-                                        w[u][1].x, w[u][1].y, w[u][1].z, w[u][1].w};
-                // (a'_0, a'_1) and (b'_0, b'_1) of the lane's pairs 2i, 2i + 1
-                float2 A[4], B[4];
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    if (kInterleaved) {
-                        A[i] = make_float2(lo_bf16(ww[2 * i]), lo_bf16(ww[2 * i + 1]));
-                        B[i] = make_float2(hi_bf16(ww[2 * i]), hi_bf16(ww[2 * i + 1]));
-                    } else {
-                        A[i] = make_float2(lo_bf16(ww[i]), hi_bf16(ww[i]));
-                        B[i] = make_float2(lo_bf16(ww[4 + i]), hi_bf16(ww[4 + i]));
-                    }
-                }
-                // a = a' c + b' s, b = b' c + a' (-s), each product and the sum rounded
-                float2 RA[4], RB[4];
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    RA[i] = sum2(mul2(A[i], C[i]), mul2(B[i], S[i]), ONE);
-                    RB[i] = sum2(mul2(B[i], C[i]), mul2(A[i], NS[i]), ONE);
-                }
-                if (n_rot < 8) {
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        if (2 * i >= n_rot) { RA[i].x = A[i].x; RB[i].x = B[i].x; }
-                        if (2 * i + 1 >= n_rot) { RA[i].y = A[i].y; RB[i].y = B[i].y; }
-                    }
-                }
-                float amax = 0.0f;
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    amax = fmaxf(amax, fabsf(RA[i].x));
-                    amax = fmaxf(amax, fabsf(RA[i].y));
-                    amax = fmaxf(amax, fabsf(RB[i].x));
-                    amax = fmaxf(amax, fabsf(RB[i].y));
-                }
-#pragma unroll
-                for (int o = kL / 2; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-                const bool fast = amax >= 0x1p-60f && amax <= 0x1p100f;
-                const float sc = fast ? div448(amax) : (amax > 0.0f ? __fdiv_rn(amax, 448.0f) : 1.0f);
-                float2 QA[4], QB[4];
-                if (fast) {
-                    // reciprocal refinement (div_by_scale), two elements per instruction
-                    const float rs = __frcp_rn(sc);
-                    const float2 RS = make_float2(rs, rs), NSC = make_float2(-sc, -sc);
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const float2 qa = mul2(RA[i], RS), qb = mul2(RB[i], RS);
-                        QA[i] = fma2(fma2(qa, NSC, RA[i]), RS, qa);
-                        QB[i] = fma2(fma2(qb, NSC, RB[i]), RS, qb);
-                    }
-                } else {
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        QA[i] = make_float2(__fdiv_rn(RA[i].x, sc), __fdiv_rn(RA[i].y, sc));
-                        QB[i] = make_float2(__fdiv_rn(RB[i].x, sc), __fdiv_rn(RB[i].y, sc));
-                    }
-                }
-                // codes in element order: chunk 0 then chunk 1
-                uint32_t c0[2], c1[2];
-                if (kInterleaved) {
-                    // elements 4i .. 4i + 3 are a_2i, b_2i, a_2i+1, b_2i+1
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const uint32_t wd = e4m3x2(QA[i].x, QB[i].x) | (e4m3x2(QA[i].y, QB[i].y) << 16);
-                        if (i < 2) c0[i] = wd;
-                        else c1[i - 2] = wd;
-                    }
-                } else {
-#pragma unroll
-                    for (int i = 0; i < 2; ++i) {
-                        c0[i] = e4m3x2(QA[2 * i].x, QA[2 * i].y) | (e4m3x2(QA[2 * i + 1].x, QA[2 * i + 1].y) << 16);
-                        c1[i] = e4m3x2(QB[2 * i].x, QB[2 * i].y) | (e4m3x2(QB[2 * i + 1].x, QB[2 * i + 1].y) << 16);
-                    }
-                }
-                if (h < h_end) {
-                    uint8_t *dst = q + (row + h) * kHd;
-                    *reinterpret_cast<uint2 *>(dst + off0) = make_uint2(c0[0], c0[1]);
-                    *reinterpret_cast<uint2 *>(dst + off1) = make_uint2(c1[0], c1[1]);
-                    if (li == 0) scales[row + h] = sc;
-                }
+                rope_head<kL, kInterleaved>(w[u][0], w[u][1], C, S, NS, ONE, n_rot, h < h_end, q + (row + h) * kHd, off0,
+                                            off1, scales + row + h, li);
             }
         }
     }
@@ -311,11 +335,11 @@ extern "C" int moe_inv_rope_quant_per_head(const moe_rope_shape_t *shape, const 
     if ((reinterpret_cast<uintptr_t>(x) & 15) || (reinterpret_cast<uintptr_t>(q) & 7) ||
         (reinterpret_cast<uintptr_t>(cos_sin) & 3) || (reinterpret_cast<uintptr_t>(scales) & 3))
         return MOE_ERR_INVALID_ARG;
+    const int L = s.head_dim / 16;
+    const int hpw = 32 / L;
     // heads per warp item: all of a token's heads when there are enough tokens
     // to give every SM 32 warps, else fewer so that small batches still spread
     // over the GPU
-    const int L = s.head_dim / 16;
-    const int hpw = 32 / L;
     int hc = s.n_heads;
     while (hc > hpw && static_cast<long long>(s.num_tokens) * ((s.n_heads + hc - 1) / hc) < 148LL * 32)
         hc = ((hc / 2) + hpw - 1) / hpw * hpw;

@@ -57,9 +57,64 @@ SMALL = [
 ]
 
 
+# Larger shapes: many warp items per resident warp, ragged head chunks
+LARGE = [
+    syn.RopeWorkload("large_partial96", T=5000, n_heads=3, head_dim=128, rot_dim=96, seed=21),
+    syn.RopeWorkload("large_il_hd256_ragged", T=2400, n_heads=20, head_dim=256, rot_dim=200, interleaved=True,
+                     seed=22),
+    syn.RopeWorkload("large_hd64_il_partial", T=2500, n_heads=40, head_dim=64, rot_dim=38, interleaved=True,
+                     seed=23),
+]
+
+
+@pytest.mark.parametrize("rw", LARGE, ids=lambda r: r.name)
+def test_inv_rope_quant_large_shapes_bit_exact(rw):
+    _check(rw, syn.rope_inputs(rw))
+
+
+def test_inv_rope_quant_large_reports_positions_out_of_range():
+    rw = syn.RopeWorkload("badpos_large", T=6000, n_heads=4, head_dim=128, rot_dim=128, max_pos=4096, seed=24)
+    d = syn.rope_inputs(rw)
+    pos = d["positions"].copy()
+    pos[[7, 4000, 5999]] = [-1, 4096, 99999]
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    q, sc = _run(rw, d, pos, status)
+    assert int(status[0]) == -5                              # MOE_ERR_DEVICE_CHECK
+    assert np.all(q[[7, 4000, 5999]] == 0) and np.all(sc[[7, 4000, 5999]] == 0)
+    rq, rs = orc.inv_rope_quant(d["x"], pos, d["cos_sin"], rw.rot_dim)
+    assert np.array_equal(q, rq) and np.array_equal(sc, rs)
+
+
 @pytest.mark.parametrize("rw", SMALL, ids=lambda r: r.name)
 def test_inv_rope_quant_shapes_bit_exact(rw):
     _check(rw, syn.rope_inputs(rw))
+
+
+@pytest.mark.parametrize("rw", [
+    syn.RopeWorkload("zeros_neox", T=40, n_heads=4, head_dim=128, rot_dim=96, seed=31),
+    syn.RopeWorkload("zeros_il", T=40, n_heads=5, head_dim=64, rot_dim=38, interleaved=True, seed=32),
+    syn.RopeWorkload("zeros_neox_large", T=5000, n_heads=3, head_dim=128, rot_dim=96, seed=33),
+    syn.RopeWorkload("zeros_il_large", T=2500, n_heads=40, head_dim=64, rot_dim=38, interleaved=True, seed=34),
+], ids=lambda r: r.name)
+def test_inv_rope_quant_signed_zero_elements(rw):
+    """Exact +0 and -0 elements inside heads of ordinary scale keep the sign
+    of their quotient (IEEE division: -0 / scale = -0, code 0x80), rotated
+    or passed through."""
+    d = syn.rope_inputs(rw)
+    x = d["x"].copy()
+    half = rw.rot_dim // 2
+    if rw.interleaved:
+        x[:, :, 0] = 0x8000; x[:, :, 1] = 0x8000          # a pair of -0
+        x[:, :, 2] = 0x8000; x[:, :, 3] = 0x0000          # -0 with a +0 partner
+    else:
+        x[:, :, 0] = 0x8000; x[:, :, half] = 0x8000
+        x[:, :, 1] = 0x8000; x[:, :, half + 1] = 0x0000
+    x[:, :, rw.rot_dim] = 0x8000                          # passed through
+    x[:, :, rw.rot_dim + 1] = 0x0000
+    d["x"] = x
+    _check(rw, d)
+    q, _ = _run(rw, d)
+    assert np.all(q[:, :, rw.rot_dim] == 0x80) and np.all(q[:, :, rw.rot_dim + 1] == 0x00)
 
 
 def test_inv_rope_quant_zero_head_and_extreme_values():
