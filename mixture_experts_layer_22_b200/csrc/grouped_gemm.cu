@@ -59,9 +59,9 @@ struct GemmParams {
     int lo_rows;             // kHiLo: row offset of the lo plane in the activation map
     int pdl;          // launched as a programmatic dependent: prefetch the first weight
                       // stages into L2 before waiting for the previous kernel
-    int rsplit;       // rows of each expert's segment: 0 all; 1 its whole 256-row
-                      // blocks; 2 the rest (under 256 rows)
-    int wait_at_end;  // the previous kernel is a launch over other rows of the same
+    int rsplit;       // which experts' segments: 0 all; 1 those of 256 rows or more;
+                      // 2 the others
+    int wait_at_end;  // the previous kernel is a launch over other experts of the same
                       // GEMM (the CTA-pair launch before an rsplit = 2 launch):
                       // nothing read here depends on it, so wait for it only before
                       // exiting, which keeps dependency waits transitive for the
@@ -286,7 +286,7 @@ __global__ void __launch_bounds__(Cfg<kMode, kSwap, kFp8, kBN, kHiLo, kPair>::kT
     using C = Cfg<kMode, kSwap, kFp8, kBN, kHiLo, kPair>;
     extern __shared__ uint8_t dyn_smem[];
     // rows [s_lo[e], s_hi[e]) of expert e's padded segment are this launch's
-    // (all of it, or with p.rsplit its whole 256-row blocks or the rest)
+    // (with p.rsplit, the whole segment or none of it)
     __shared__ int s_lo[kMaxExpertsTotal], s_hi[kMaxExpertsTotal];
     __shared__ int s_prefix[kMaxExpertsTotal + 1];
     __shared__ __align__(8) uint64_t s_full[C::kSlots], s_empty[C::kSlots];
@@ -357,9 +357,9 @@ __global__ void __launch_bounds__(Cfg<kMode, kSwap, kFp8, kBN, kHiLo, kPair>::kT
         for (int e = lane; e < Et; e += 32) {
             const int a = __ldcg(p.offsets + e), b = __ldcg(p.offsets + e + 1);
             if (b < a || ((b - a) & 15) != 0 || (a & 15) != 0) bad = true;
-            const int blocks = b > a ? a + (b - a) / 256 * 256 : a;   // end of the whole 256-row blocks
-            s_lo[e] = p.rsplit == 2 ? blocks : a;
-            s_hi[e] = p.rsplit == 1 ? blocks : b;
+            const bool big = b - a >= 256;
+            s_lo[e] = a;
+            s_hi[e] = p.rsplit == 0 ? b : (p.rsplit == 1 ? (big ? b : a) : (big ? a : b));
         }
         __syncwarp();
         const int per = (Et + 31) / 32;
@@ -1338,13 +1338,14 @@ cudaError_t launch_grouped_gemm(const moe_shape_t &s, const GemmPlan &p, const G
             if (fp8) { MOE_BY_BN(1, true) } else { MOE_BY_BN(1, false) }
         }
     } else {
-        // Normal order (prefill).  Each expert's whole 256-row blocks run on
-        // CTA pairs (256 x 256 tiles, half the weight bytes staged per SM),
-        // then the rest of its segment (under 256 rows) on one-CTA 128-row
-        // tiles, which pad at most 127 rows per expert where a pair tile pads
-        // up to 255.  The second launch reads nothing the first writes: it
-        // starts as the pairs' SMs free up and waits for them only before
-        // exiting.
+        // Normal order (prefill).  Experts with 256 rows or more run on CTA
+        // pairs (256 x 256 tiles, half the weight bytes staged per SM), the
+        // others on one-CTA 128-row tiles in a second launch, which pads at
+        // most 127 rows per expert where a pair tile pads up to 255.  Each
+        // expert's weights are read by one launch only (splitting a segment
+        // between the two launches read its weights twice from HBM).  The
+        // second launch reads nothing the first writes: it starts as the
+        // pairs' SMs free up and waits for them only before exiting.
         GemmArgs g = a;
         g.rsplit = 1;
         if (a.mode == 0) {
