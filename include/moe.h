@@ -320,6 +320,23 @@ int moe_inv_rope_quant_per_head(const moe_rope_shape_t *shape, const void *x, co
 int moe_selftest_wait_timeout(void *ws, int32_t *gave_up, moe_stream_t stream);
 
 /*
+ * Self-test of the CTA-pair abort path (no counterpart on the pages): the
+ * down projection of moe_grouped_gemm_down (same arguments; bf16 weights and
+ * activations, a shape on the normal order: more than 128 tokens, or
+ * variant MOE_VARIANT_NORMAL), except that in every CTA pair the second CTA
+ * stops loading its half of the operands after two stages.  The first CTA's
+ * waits for those stages run out after the wait limit (2 s); both CTAs then
+ * take the pair's abort tear-down (no copy left in flight into either CTA,
+ * tensor memory freed), MOE_ERR_TIMEOUT goes to the status word at the start
+ * of `ws`, and the kernel exits, so the CUDA context stays usable.  The
+ * experts handled by one-CTA tiles are computed normally; y of the experts
+ * on pairs is undefined.  Returns MOE_ERR_UNSUPPORTED for other shapes.
+ * Asynchronous on `stream`.
+ */
+int moe_selftest_pair_abort(const moe_shape_t *shape, const void *h, const void *w2, const int32_t *offsets,
+                            float *y, void *ws, size_t ws_bytes, moe_stream_t stream);
+
+/*
  * Device status written by the kernels into `ws`: copies it to *status
  * (host) after synchronising `stream` -- the one call here that waits.
  * MOE_OK when no kernel reported a problem since the last reset.

@@ -30,7 +30,8 @@ EXPORTS = ["moe_max_rows", "moe_workspace_size", "moe_route_topk", "moe_align_pe
            "moe_grouped_gemm_swiglu", "moe_grouped_gemm_down", "moe_combine", "moe_fused_forward",
            "moe_get_device_status", "moe_reset_device_status", "moe_status_string",
            "moe_last_launch_count", "moe_align_permute_noalloc", "moe_router_topk",
-           "moe_fused_forward_router", "moe_selftest_wait_timeout", "moe_inv_rope_quant_per_head"]
+           "moe_fused_forward_router", "moe_selftest_wait_timeout", "moe_selftest_pair_abort",
+           "moe_inv_rope_quant_per_head"]
 
 
 class MoeError(RuntimeError):
@@ -94,6 +95,7 @@ def lib() -> C.CDLL:
             "moe_router_topk": [S, P, P, P, P, P, P, C.c_size_t, P],
             "moe_fused_forward_router": [S, P, P, P, P, P, P, C.c_float, C.c_float, P, P, C.c_size_t, P],
             "moe_selftest_wait_timeout": [P, P, P],
+            "moe_selftest_pair_abort": [S, P, P, P, P, P, C.c_size_t, P],
             "moe_inv_rope_quant_per_head": [C.POINTER(RopeShape), P, P, P, P, P, P, P],
         }
         for name, args in sig.items():
@@ -225,6 +227,14 @@ def selftest_wait_timeout(ws, gave_up, stream=None):
     """Launch the failure-path self-test (about 2 s on the GPU): its bounded
     waits run out and it reports MOE_ERR_TIMEOUT in ws's status word."""
     _check(lib().moe_selftest_wait_timeout(_ptr(ws), _ptr(gave_up), _stream(stream)), "moe_selftest_wait_timeout")
+
+
+def selftest_pair_abort(shape, h, w2, offsets, y, ws, stream=None):
+    """The down projection with the second CTA of every CTA pair stalled
+    (about 2 s on the GPU): the pairs' waits run out, they take their abort
+    tear-down and MOE_ERR_TIMEOUT goes to ws's status word."""
+    _check(lib().moe_selftest_pair_abort(C.byref(shape), _ptr(h), _ptr(w2), _ptr(offsets), _ptr(y), _ptr(ws),
+                                         ws.numel(), _stream(stream)), "moe_selftest_pair_abort")
 
 
 def device_status(ws, stream=None) -> int:

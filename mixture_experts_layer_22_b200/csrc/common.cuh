@@ -212,6 +212,7 @@ struct GemmArgs {
     // normal order: which rows of each segment this launch takes (GemmParams)
     int rsplit = 0;
     bool wait_at_end = false;
+    int test_stall = 0;       // abort-path test only (GemmParams::test_stall)
 };
 cudaError_t launch_grouped_gemm(const moe_shape_t &s, const GemmPlan &p, const GemmArgs &a,
                                 cudaStream_t st, int *launches, int *host_err);

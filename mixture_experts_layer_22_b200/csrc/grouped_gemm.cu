@@ -61,6 +61,9 @@ struct GemmParams {
                       // stages into L2 before waiting for the previous kernel
     int rsplit;       // which experts' segments: 0 all; 1 those of 256 rows or more;
                       // 2 the others
+    int test_stall;   // test of the abort path only (0 otherwise): in a CTA pair, rank
+                      // 1's producer stops after this many stage fills, so that rank
+                      // 0's waits run out and the pair's abort tear-down runs
     int wait_at_end;  // the previous kernel is a launch over other experts of the same
                       // GEMM (the CTA-pair launch before an rsplit = 2 launch):
                       // nothing read here depends on it, so wait for it only before
@@ -483,6 +486,10 @@ __global__ void __launch_bounds__(Cfg<kMode, kSwap, kFp8, kBN, kHiLo, kPair>::kT
                 const int rows = min(C::kRowsTile, s_hi[it.e] - row0);
                 const int wbase = it.e * p.w_rows;
                 for (int kk = it.kb; kk < it.ke; ++kk) {
+                    if (kPair && p.test_stall > 0 && rank == 1 && in_flight >= p.test_stall) {
+                        ok = false;
+                        break;
+                    }
                     if (!mbar_wait(smem_u32(&s_empty[stage]), phase ^ 1u, &s_abort)) {
                         ok = false;
                         break;
@@ -1246,6 +1253,7 @@ static cudaError_t run_gemm(const moe_shape_t &s, const GemmArgs &a, cudaStream_
     p.next_reverse = a.next_reverse ? 1 : 0;
     p.rsplit = a.rsplit;
     p.wait_at_end = a.wait_at_end ? 1 : 0;
+    p.test_stall = kPair ? a.test_stall : 0;
     // When to split tiles.  Decode (Swap-AB): above 3% idle, unless the idle
     // work is under 12 K-steps per CTA.  A split item's epilogue (partial
     // store, fixup, combine) costs about that much of the weight stream: on
@@ -1357,6 +1365,7 @@ cudaError_t launch_grouped_gemm(const moe_shape_t &s, const GemmPlan &p, const G
         }
         if (err != cudaSuccess || *host_err != MOE_OK) return err;
         *launches += 1;
+        g.test_stall = 0;
         g.rsplit = 2;
         g.chained = true;
         g.wait_at_end = true;

@@ -206,7 +206,7 @@ int moe_gather(const moe_shape_t *shape, const void *x, const int32_t *sorted_ro
 
 static int gemm_common(const moe_shape_t *shape, int mode, const void *act, const void *wgt,
                        const float *wscale, float ascale, float qscale, const int32_t *offsets,
-                       void *out, void *ws, size_t ws_bytes, cudaStream_t stream)
+                       void *out, void *ws, size_t ws_bytes, cudaStream_t stream, int test_stall = 0)
 {
     int st = validate_shape(shape, true);
     if (st != MOE_OK) return st;
@@ -235,6 +235,7 @@ static int gemm_common(const moe_shape_t *shape, int mode, const void *act, cons
     a.planes = b + L.planes;
     a.rowscale = reinterpret_cast<float *>(b + L.rowscale);
     a.max_rows = L.max_rows;
+    a.test_stall = test_stall;
     int host_err = MOE_OK;
     cudaError_t e = launch_grouped_gemm(*shape, plan_gemm(*shape), a, stream, &g_launches, &host_err);
     if (host_err != MOE_OK) return host_err;
@@ -258,6 +259,16 @@ int moe_grouped_gemm_down(const moe_shape_t *shape, const void *h, const void *w
     g_launches = 0;
     return gemm_common(shape, 1, h, w2, w2_scale, a2_scale, a2_scale, offsets, y, ws, ws_bytes,
                        reinterpret_cast<cudaStream_t>(stream));
+}
+
+int moe_selftest_pair_abort(const moe_shape_t *shape, const void *h, const void *w2, const int32_t *offsets,
+                            float *y, void *ws, size_t ws_bytes, moe_stream_t stream)
+{
+    g_launches = 0;
+    if (!shape || plan_gemm(*shape).swap || shape->wdtype != MOE_BF16 || shape->adtype != MOE_BF16)
+        return MOE_ERR_UNSUPPORTED;
+    return gemm_common(shape, 1, h, w2, nullptr, 1.0f, 1.0f, offsets, y, ws, ws_bytes,
+                       reinterpret_cast<cudaStream_t>(stream), 2);
 }
 
 int moe_combine(const moe_shape_t *shape, const float *y, const float *w, const int32_t *inv,

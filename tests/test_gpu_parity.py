@@ -479,11 +479,51 @@ def test_bounded_wait_times_out_and_context_stays_usable():
     assert rel_err(got, oracle_forward(wl, d), "bf16") <= BF16_TOL
 
 
-# ------------------------------------------------------------------ fused gather and combine
-# The fused layer gathers GEMM1's token rows straight from x (tile::gather4)
-# and combines inside GEMM2's epilogue.  The arithmetic and its order are
-# those of the separate steps, so the fused output must equal, bit for bit,
-# the output of the step-by-step calls on the same inputs.
+def test_cta_pair_abort_times_out_and_context_stays_usable():
+    """In every CTA pair of a prefill down projection the second CTA stops
+    loading its operand halves after two stages.  The first CTA's waits run
+    out after the wait limit, both CTAs take the pair's abort tear-down (no
+    copy left in flight, tensor memory freed), the status word reads
+    MOE_ERR_TIMEOUT, the call ends within seconds, and the next layer call on
+    the same context is correct."""
+    import time
+    wl = W["tiny"].with_T(2048)            # 4096 routed rows over 8 experts: all on CTA pairs
+    d = syn.make_inputs(wl)
+    L = Layer(wl, d)
+    s = L.shape
+    E_t = wl.E + wl.n_shared
+    mr = moe.max_rows(s)
+    ids = torch.empty((wl.T, wl.k), dtype=torch.int32, device="cuda")
+    w = torch.empty((wl.T, wl.k), dtype=torch.float32, device="cuda")
+    counts = torch.empty(E_t, dtype=torch.int32, device="cuda")
+    offsets = torch.empty(E_t + 1, dtype=torch.int32, device="cuda")
+    rows = torch.empty(mr, dtype=torch.int32, device="cuda")
+    inv = torch.empty(wl.T * wl.k, dtype=torch.int32, device="cuda")
+    h = torch.zeros((mr, wl.I), dtype=torch.bfloat16, device="cuda")
+    y = torch.empty((mr, wl.H), dtype=torch.float32, device="cuda")
+    ws = moe.workspace(s)
+    moe.reset_device_status(ws)
+    moe.route_topk(s, L.logits, ids, w)
+    moe.align_permute(s, ids, counts, offsets, rows, inv, ws)
+    torch.cuda.synchronize()
+    assert int(counts.min()) >= 256                       # every expert's segment goes to the pairs
+    t0 = time.perf_counter()
+    moe.selftest_pair_abort(s, h, L.w2, offsets, y, ws)
+    torch.cuda.synchronize()
+    dt = time.perf_counter() - t0
+    assert moe.device_status(ws) == -6                     # MOE_ERR_TIMEOUT
+    assert 1.5 < dt < 30.0
+    got = L.run()                                          # resets the status, runs the layer
+    assert L.status() == 0
+    assert rel_err(got, oracle_forward(wl, d), "bf16") <= BF16_TOL
+
+
+# ------------------------------------------------------------------ fused layer against the separate steps
+# The fused layer routes and aligns in one kernel at decode sizes, skips pad
+# slots, and combines inside GEMM2's epilogue on the Swap-AB path.  The
+# arithmetic and its order are those of the separate steps, so the fused
+# output must equal, bit for bit, the output of the step-by-step calls on the
+# same inputs.
 STEPWISE = [
     (W["tiny"], moe.SWAP_AB), (W["tiny"], moe.NORMAL),
     (EDGE[0], moe.SWAP_AB), (EDGE[0], moe.NORMAL),                  # ragged T=37
