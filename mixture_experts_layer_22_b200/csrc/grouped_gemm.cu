@@ -672,7 +672,7 @@ __global__ void __launch_bounds__(Cfg<kMode, kSwap, kFp8, kBN, kHiLo, kPair>::kT
             const float sc = (kHiLo ? 1.0f : p.ascale) * (p.wscale ? __ldg(&p.wscale[it.e]) : 1.0f);
             // fused combine: each row's staging row and token (-1 for pad
             // slots), a per-tile table filled by all epilogue threads before use
-            if constexpr (kMode == 1) {
+            if constexpr (kMode == 1 && kSwap) {
                 for (int i = etid; p.combine && i < rows; i += C::kEpiThreads) {
                     const int code = __ldg(p.sorted_rows + row0 + i);
                     int t = -1, dst = -1;
@@ -724,10 +724,9 @@ __global__ void __launch_bounds__(Cfg<kMode, kSwap, kFp8, kBN, kHiLo, kPair>::kT
                 const int ngrp = min(fcols, p.n_feat - h0) / 4;      // 4-feature groups
                 const int items = nf * ngrp;
                 // rows of a token prefetched per item (the rest load in order) and
-                // items per thread at a time: the 192-thread Swap-AB kernels have
-                // registers to spare, the 320-thread CTA-pair ones do not
+                // items per thread at a time
                 constexpr int kU = 2;
-                constexpr int kMaxS = kSwap ? 9 : 4;
+                constexpr int kMaxS = 9;
                 for (int base = etid; base < items; base += kU * C::kEpiThreads) {
                     float4 v[kU][kMaxS];
                     int tk[kU], g4[kU];
@@ -908,13 +907,9 @@ __global__ void __launch_bounds__(Cfg<kMode, kSwap, kFp8, kBN, kHiLo, kPair>::kT
                             const int rl = ps * 8 + (lane >> 2);
                             const int rg = q * 32 + rl;
                             const float4 val = *reinterpret_cast<const float4 *>(stg + rl * kStagePitch + (lane & 3) * 16);
-                            if (rg < rows) {
-                                const int dr = p.combine ? s_dst[rg] : row0 + rg;
-                                float *dstp = p.combine ? p.ystage : static_cast<float *>(p.out);
-                                if (dr >= 0)
-                                    *reinterpret_cast<float4 *>(dstp + static_cast<size_t>(dr) * p.out_ld + h0 + c0 + (lane & 3) * 4) =
-                                        val;
-                            }
+                            if (rg < rows)
+                                *reinterpret_cast<float4 *>(static_cast<float *>(p.out) +
+                                                            static_cast<size_t>(row0 + rg) * p.out_ld + h0 + c0 + (lane & 3) * 4) = val;
                         }
                         __syncwarp();
                     }
@@ -926,10 +921,11 @@ __global__ void __launch_bounds__(Cfg<kMode, kSwap, kFp8, kBN, kHiLo, kPair>::kT
                     if constexpr (kPair) mbar_arrive_cluster(mapa_shared(smem_u32(&s_tempty[acc]), 0));
                     else mbar_arrive(smem_u32(&s_tempty[acc]));
                 }
-                if constexpr (kMode == 1)
-                    if (p.combine) combine_tail(rows, it.ft * (kSwap ? 128 : 256), kSwap ? 128 : 256);
-            } else {
+                if constexpr (kMode == 1 && kSwap)
+                    if (p.combine) combine_tail(rows, it.ft * 128, 128);
+            } else if constexpr (kSwap) {
                 // ---- one share of a split tile: store the raw partial ----
+                // (decode only: prefill launches take whole tiles)
                 float *slot = p.partials + static_cast<size_t>(it.slot) * 128 * C::kAccCols;
                 for (int c0 = ch * (ncols / kNch); c0 < (ch + 1) * (ncols / kNch); c0 += 16) {
                     uint32_t v[16];
@@ -991,35 +987,6 @@ __global__ void __launch_bounds__(Cfg<kMode, kSwap, kFp8, kBN, kHiLo, kPair>::kT
                         }
                         if constexpr (kMode == 1)
                             if (p.combine) combine_tail(ncols, h0, 128);
-                    } else if (kMode == 0) {
-                        const int f0 = it.ft * 128;
-                        const int rr = etid & 127, hf = etid >> 7;
-                        if (rr < rows)
-                            for (int j = hf * (128 / kNch); j < (hf + 1) * (128 / kNch); ++j) {
-                                float g = 0.f, u = 0.f;
-                                for (int c = c_first; c <= c_last; ++c) {
-                                    const float *ps = slot_of(c);
-                                    g += __ldcg(&ps[j * 128 + rr]);
-                                    u += __ldcg(&ps[(128 + j) * 128 + rr]);
-                                }
-                                const float hv = silu_mul(g * sc, u * sc);
-                                const size_t o = static_cast<size_t>(row0 + rr) * p.out_ld + f0 + j;
-                                if (C::kOutE4M3) static_cast<uint8_t *>(p.out)[o] = static_cast<uint8_t>(e4m3_code(hv / p.qscale));
-                                else static_cast<__nv_bfloat16 *>(p.out)[o] = __float2bfloat16_rn(hv);
-                            }
-                    } else {
-                        const int h0 = it.ft * 256;
-                        const int rr = etid & 127, hf = etid >> 7;
-                        const int dr = rr < rows ? (p.combine ? s_dst[rr] : row0 + rr) : -1;
-                        float *dstp = p.combine ? p.ystage : static_cast<float *>(p.out);
-                        if (dr >= 0)
-                            for (int j = hf * (256 / kNch); j < (hf + 1) * (256 / kNch) && h0 + j < p.n_feat; ++j) {
-                                float a = 0.f;
-                                for (int c = c_first; c <= c_last; ++c) a += __ldcg(&slot_of(c)[j * 128 + rr]);
-                                dstp[static_cast<size_t>(dr) * p.out_ld + h0 + j] = a * sc;
-                            }
-                        if constexpr (kMode == 1)
-                            if (p.combine) combine_tail(rows, h0, 256);
                     }
                 }
                 named_bar_sync(1, C::kEpiThreads);
@@ -1241,7 +1208,7 @@ static cudaError_t run_gemm(const moe_shape_t &s, const GemmArgs &a, cudaStream_
     p.k = s.k;
     p.R = s.T * s.k;
     p.n_shared = s.n_shared;
-    p.combine = kMode == 1 && a.combine ? 1 : 0;
+    p.combine = kMode == 1 && kSwap && a.combine ? 1 : 0;   // the combine is fused on the Swap-AB path only
     p.ystage = a.ystage;
     p.tok_cnt = a.tok_cnt;
     p.n_ct = (s.H + (kSwap ? 127 : 255)) / (kSwap ? 128 : 256);
