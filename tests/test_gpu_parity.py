@@ -328,6 +328,40 @@ def test_fused_edge_cases(wl, pad):
         assert rel_err(got, ref, "bf16") <= BF16_TOL, (variant, pad)
 
 
+def _random_shapes(n=16, seed=7):
+    """Seeded random layer shapes across the supported space (H, I multiples
+    of 128; ragged T; 1 to 64 experts; top-1 to top-8; softmax or sigmoid
+    gate; a shared expert or none; bf16 or E4M3 weights; both operand
+    orders).  The list is fixed by the seed, so a failure names its shape."""
+    rng = np.random.default_rng(seed)
+    out = []
+    for i in range(n):
+        E = int(rng.choice([1, 2, 5, 8, 16, 33, 64]))
+        k = int(rng.integers(1, min(E, 8) + 1))
+        w8 = bool(rng.random() < 0.25)
+        wl = syn.Workload(f"rand{i}", T=int(rng.integers(1, 700)), H=int(rng.choice([128, 256, 384, 640])),
+                          I=int(rng.choice([128, 256, 512, 896])), E=E, k=k,
+                          n_shared=int(rng.random() < 0.3),
+                          gate=syn.SIGMOID if rng.random() < 0.3 else syn.SOFTMAX,
+                          routed_scale=float(rng.choice([1.0, 2.5])),
+                          wdtype=syn.E4M3 if w8 else syn.BF16, seed=100 + i)
+        variant = moe.SWAP_AB if w8 else [moe.AUTO, moe.SWAP_AB, moe.NORMAL][int(rng.integers(0, 3))]
+        pad = int(rng.choice([16, 32, 64]))
+        out.append((wl, variant, pad))
+    return out
+
+
+@pytest.mark.parametrize("wl,variant,pad", _random_shapes(),
+                         ids=lambda v: getattr(v, "name", str(v)))
+def test_fused_random_shapes(wl, variant, pad):
+    d = syn.make_inputs(wl)
+    ref = oracle_forward(wl, d)
+    L = Layer(wl, d, pad=pad, variant=variant)
+    got = L.run()
+    assert L.status() == 0
+    assert rel_err(got, ref, "bf16") <= BF16_TOL, (wl, variant, pad)
+
+
 def _fp8_small(T=300):
     wl = syn.Workload("fp8_small", T=T, H=512, I=512, E=8, k=2, wdtype=syn.E4M3, adtype=syn.E4M3, seed=7)
     d = syn.make_inputs(wl)
