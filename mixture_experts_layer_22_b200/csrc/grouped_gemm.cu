@@ -135,7 +135,7 @@ struct Cfg {
     static constexpr bool kOutE4M3 = kFp8 && !kHiLo;
     static_assert(kStages >= 2, "smem ring too small");
     static_assert(!kSwap || kRingBytes >= 2 * kStage, "Swap-AB ring must hold two full-size stages");
-    static_assert(!kHiLo || (kSwap && kFp8 && kBN <= 128), "hi/lo planes: Swap-AB on the E4M3 tensor path");
+    static_assert(!kHiLo || (kSwap && kFp8 && kBN == 16), "hi/lo planes: Swap-AB on the E4M3 tensor path, 16-row tiles");
     // kPair: normal order on a CTA pair (tcgen05 .cta_group::2): M = 256 token
     // rows (128 per CTA), N = 256 weight rows (each CTA stages its 128), each
     // CTA's tensor memory holds its 128 rows x 256 columns
@@ -452,6 +452,8 @@ __global__ void __launch_bounds__(Cfg<kMode, kSwap, kFp8, kBN, kHiLo, kPair>::kT
                     // this CTA's half: gate (rank 0) or up (rank 1) rows; W2 rows [128 rank, +128)
                     tma_prefetch_l2_2d(&tm_w, kx, kMode == 0 ? wbase + (rank ? p.n_feat : 0) + it.ft * 128
                                                              : wbase + it.ft * 256 + 128 * static_cast<int>(rank));
+                } else if (kMode == 0 && kSwap) {
+                    tma_prefetch_l2_4d(&tm_w, kx, it.ft * kHalf, 0, it.e);
                 } else if (kMode == 0) {
                     tma_prefetch_l2_2d(&tm_w, kx, wbase + it.ft * kHalf);
                     tma_prefetch_l2_2d(&tm_w, kx, wbase + p.n_feat + it.ft * kHalf);
@@ -505,17 +507,18 @@ __global__ void __launch_bounds__(Cfg<kMode, kSwap, kFp8, kBN, kHiLo, kPair>::kT
                     const uint32_t sb = sa + C::kStageA;
                     const int kx = kk * C::kKStage;
                     if (kSwap) {
-                        if (kMode == 0) {
-                            tma_load_2d(sa, &tm_w, fb, kx, wbase + it.ft * 64, pol_w);
-                            tma_load_2d(sa + 64 * C::kRowBytes, &tm_w, fb, kx, wbase + p.n_feat + it.ft * 64, pol_w);
-                        } else {
+                        // one instruction per operand where the layout allows:
+                        // the single producer thread's work per stage bounds
+                        // the weight stream
+                        if (kMode == 0)   // the expert's 64 gate rows, then its 64 up rows (4-D map)
+                            tma_load_4d(sa, &tm_w, fb, kx, it.ft * 64, 0, it.e, pol_w);
+                        else
                             tma_load_2d(sa, &tm_w, fb, kx, wbase + it.ft * 128, pol_w);
-                        }
-                        for (int rr = 0; rr < rows; rr += 16)
-                            tma_load_2d(sb + rr * C::kRowBytes, &tm_x, fb, kx, row0 + rr, pol_x);
-                        if (kHiLo)
+                        if (kHiLo)        // 16 token rows of the hi plane, then of the lo plane (3-D map)
+                            tma_load_3d(sb, &tm_x, fb, kx, row0, 0, pol_x);
+                        else
                             for (int rr = 0; rr < rows; rr += 16)
-                                tma_load_2d(sb + (rows + rr) * C::kRowBytes, &tm_x, fb, kx, p.lo_rows + row0 + rr, pol_x);
+                                tma_load_2d(sb + rr * C::kRowBytes, &tm_x, fb, kx, row0 + rr, pol_x);
                     } else if (kPair) {
                         // this CTA's 128 token rows and its half of the 256 weight
                         // rows (gate or up rows of 128 features; W2 rows [128 rank, +128))
@@ -1059,18 +1062,21 @@ static EncodeTiledFn get_encode_fn()
     return fn;
 }
 
-// 2-D map over a row-major [rows, cols] matrix with 128-byte rows per box
-// and the 128-byte swizzle; box = box_rows x (128 bytes).  A map depends only
-// on these arguments (not on the device or on what the memory holds), so the
-// last few are kept per host thread and a repeat call with the same buffers
-// skips the encode.
-static bool make_map(CUtensorMap *m, const void *base, bool u8, uint64_t rows, uint64_t cols,
-                     uint32_t box_rows)
+// Map over a row-major tensor of 2 to 4 dimensions (dims[0] the contiguous
+// one) with the 128-byte swizzle; a box is 128 bytes of dims[0] times box[1..]
+// of the others.  A map depends only on these arguments (not on the device
+// or on what the memory holds), so the last few are kept per host thread and
+// a repeat call with the same buffers skips the encode.
+static bool make_map_nd(CUtensorMap *m, const void *base, bool u8, int rank, const uint64_t *dims,
+                        const uint32_t *box)
 {
+    // dims[0] = cols (elements, contiguous), dims[1..] row-major outer extents;
+    // box[0] is implied (128 bytes of cols)
     struct Entry {
         const void *base;
-        uint64_t rows, cols;
-        uint32_t box_rows;
+        int rank;
+        uint64_t dims[4];
+        uint32_t box[4];
         bool u8, valid;
         CUtensorMap map;
     };
@@ -1079,7 +1085,9 @@ static bool make_map(CUtensorMap *m, const void *base, bool u8, uint64_t rows, u
     thread_local int next = 0;
     for (int i = 0; i < kEntries; ++i) {
         const Entry &c = cache[i];
-        if (c.valid && c.base == base && c.rows == rows && c.cols == cols && c.box_rows == box_rows && c.u8 == u8) {
+        bool same = c.valid && c.base == base && c.rank == rank && c.u8 == u8;
+        for (int d = 0; same && d < rank; ++d) same = c.dims[d] == dims[d] && (d == 0 || c.box[d] == box[d]);
+        if (same) {
             *m = c.map;
             return true;
         }
@@ -1088,20 +1096,39 @@ static bool make_map(CUtensorMap *m, const void *base, bool u8, uint64_t rows, u
     EncodeTiledFn fn = get_encode_fn();
     if (!fn) return false;
     const uint32_t esz = u8 ? 1 : 2;
-    cuuint64_t dims[2] = {cols, rows};
-    cuuint64_t strides[1] = {cols * esz};
-    cuuint32_t box[2] = {row_bytes / esz, box_rows};
-    cuuint32_t estr[2] = {1, 1};
-    CUresult r = fn(m, u8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
-                    const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                    CU_TENSOR_MAP_SWIZZLE_128B,
-                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+    cuuint64_t gdims[4], strides[3];
+    cuuint32_t gbox[4], estr[4] = {1, 1, 1, 1};
+    uint64_t pitch = dims[0] * esz;
+    for (int d = 0; d < rank; ++d) {
+        gdims[d] = dims[d];
+        gbox[d] = d == 0 ? row_bytes / esz : box[d];
+        if (d > 0) {
+            strides[d - 1] = pitch;
+            pitch *= dims[d];
+        }
+    }
+    CUresult r = fn(m, u8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                    static_cast<cuuint32_t>(rank), const_cast<void *>(base), gdims, strides, gbox, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return false;
     Entry &c = cache[next];
     next = (next + 1) % kEntries;
-    c = Entry{base, rows, cols, box_rows, u8, true, *m};
+    c = Entry{base, rank, {0, 0, 0, 0}, {0, 0, 0, 0}, u8, true, *m};
+    for (int d = 0; d < rank; ++d) {
+        c.dims[d] = dims[d];
+        c.box[d] = box[d];
+    }
     return true;
+}
+
+// 2-D map over a row-major [rows, cols] matrix with 128-byte rows per box
+// and the 128-byte swizzle; box = box_rows x (128 bytes).
+static bool make_map(CUtensorMap *m, const void *base, bool u8, uint64_t rows, uint64_t cols, uint32_t box_rows)
+{
+    const uint64_t dims[2] = {cols, rows};
+    const uint32_t box[2] = {0, box_rows};
+    return make_map_nd(m, base, u8, 2, dims, box);
 }
 
 // SMs of the current device (the persistent grid size), cached per device.
@@ -1171,8 +1198,18 @@ static cudaError_t run_gemm(const moe_shape_t &s, const GemmArgs &a, cudaStream_
     const uint32_t xbox = kSwap ? 16 : 128;     // Swap-AB loads token rows in 16-row boxes
     CUtensorMap tm_w, tm_x, tm_next;
     static_assert(Cf::kRowBytes == 128, "tensor maps use 128-byte rows with the 128-byte swizzle");
-    if (!make_map(&tm_w, a.wgt, u8w, Et * w_rows, K, wbox) ||
-        !make_map(&tm_x, a.act, u8, Cf::kPlanes * a.max_rows, K, xbox)) {
+    // Swap-AB gate/up: [Et][2][I][H] as 4-D, one box = an expert's 64 gate
+    // rows and 64 up rows; hi/lo activations: [2][max_rows][K] as 3-D, one
+    // box = 16 rows of both planes
+    const uint64_t wdims[4] = {static_cast<uint64_t>(K), static_cast<uint64_t>(s.I), 2, static_cast<uint64_t>(Et)};
+    const uint32_t wbox4[4] = {0, 64, 2, 1};
+    const uint64_t xdims[3] = {static_cast<uint64_t>(K), static_cast<uint64_t>(a.max_rows), 2};
+    const uint32_t xbox3[3] = {0, 16, 2};
+    const bool w_ok = kSwap && kMode == 0 ? make_map_nd(&tm_w, a.wgt, u8w, 4, wdims, wbox4)
+                                          : make_map(&tm_w, a.wgt, u8w, Et * w_rows, K, wbox);
+    const bool x_ok = kHiLo ? make_map_nd(&tm_x, a.act, u8, 3, xdims, xbox3)
+                            : make_map(&tm_x, a.act, u8, Cf::kPlanes * a.max_rows, K, xbox);
+    if (!w_ok || !x_ok) {
         *host_err = MOE_ERR_CUDA;
         return cudaSuccess;
     }
@@ -1285,14 +1322,9 @@ cudaError_t launch_grouped_gemm(const moe_shape_t &s, const GemmPlan &p, const G
         }
         g.act = a.planes;
 #define MOE_W8(MODE, BN) err = run_gemm<MODE, true, true, BN, true>(s, g, st, host_err)
-#define MOE_W8_BY_BN(MODE)                   \
-    switch (p.bn) {                          \
-    case 16: MOE_W8(MODE, 16); break;        \
-    case 32: MOE_W8(MODE, 32); break;        \
-    default: MOE_W8(MODE, 64); break;        \
-    }
-        if (a.mode == 0) { MOE_W8_BY_BN(0) } else { MOE_W8_BY_BN(1) }
-#undef MOE_W8_BY_BN
+        // hi/lo tiles take 16 token rows (plan_gemm)
+        if (a.mode == 0) MOE_W8(0, 16);
+        else MOE_W8(1, 16);
 #undef MOE_W8
         *launches += 1;
         return err;

@@ -48,15 +48,17 @@ GemmPlan plan_gemm(const moe_shape_t &s)
     if (p.swap) {
         const int rows = (s.T + s.pad - 1) / s.pad * s.pad;   // worst case rows of one expert
         int bn = 16;
-        // The hi/lo path holds two planes per token row, so a 64-row tile
-        // already stages and accumulates 128 columns.  The smem ring is sized
-        // per launch from the largest segment (the shared expert's T rows at
-        // T >= 64), and 64-row tiles keep 6 stages in flight where 128-row
-        // ones would keep 4 for the whole weight stream.  The price is that a
-        // segment of more than 64 rows takes two row tiles over the same
-        // weight tile; those are adjacent in the tile list, so they run at the
-        // same time and the second read comes mostly from L2.
-        const int cap = (s.wdtype == MOE_E4M3 && s.adtype == MOE_BF16) ? 64 : 256;
+        // The hi/lo path holds two planes per token row in every stage, and
+        // the smem ring is sized per launch from the largest segment (the
+        // shared expert's T rows).  Its weight stream is bound by how many
+        // bytes each SM keeps in flight, so its tiles take 16 rows: 20 KB
+        // stages, 10 in the ring, where 64-row tiles (32 KB stages) kept 6
+        // for every expert because of the shared one (measured 3-4% faster at
+        // T = 32..128).  The price is that a segment of more than 16 rows
+        // takes several row tiles over the same weight tile; those are
+        // adjacent in the tile list, so they run at the same time and the
+        // repeat reads come from L2.
+        const int cap = (s.wdtype == MOE_E4M3 && s.adtype == MOE_BF16) ? 16 : 256;
         while (bn < rows && bn < cap) bn <<= 1;
         p.bn = bn;
     } else {
