@@ -383,10 +383,37 @@ class DeviceLayer:
         return 1e6 * (t1 - t0) / n
 
 
-def time_steps(L, steps, graph, flush=None):
+class L2Flush:
+    """Empties L2 between timed steps, outside the timed intervals: a 256 MB
+    buffer (twice L2) is written, which evicts the step's data, and then, with
+    `clean`, a second 256 MB buffer is read.  The read makes L2 write back the
+    first buffer's dirty lines before the timed step starts; without it the
+    step would begin by writing back up to 126 MB that are not its own."""
+
+    MB = 256
+
+    def __init__(self, torch, dev):
+        n = self.MB * 2 ** 20 // 4
+        self.torch = torch
+        self.w = torch.empty(n, dtype=torch.float32, device=dev)
+        self.r = torch.zeros(n, dtype=torch.float32, device=dev)
+        self.s = torch.empty((), dtype=torch.float32, device=dev)
+
+    def __call__(self, stream, clean=True):
+        with self.torch.cuda.stream(stream):
+            self.w.add_(1)
+            if clean:
+                self.torch.sum(self.r, dim=0, out=self.s)
+
+    def describe(self, clean=True):
+        return (f"flushed between timed steps: {self.MB} MB written" +
+                (f", then {self.MB} MB read (no dirty lines left in L2)" if clean else " (L2 left dirty)"))
+
+
+def time_steps(L, steps, graph, flush=None, clean=True):
     """Device milliseconds of `steps` layer steps on L's stream.  With `flush`
-    (a buffer larger than L2) each step is timed alone and L2 is rewritten
-    between steps, outside the timed intervals."""
+    (an L2Flush) each step is timed alone and L2 is emptied between steps,
+    outside the timed intervals."""
     torch = L.torch
     st = L.stream
     if flush is None:
@@ -399,8 +426,7 @@ def time_steps(L, steps, graph, flush=None):
         return e0.elapsed_time(e1)
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
     for a, b in ev:
-        with torch.cuda.stream(st):
-            flush.add_(1)
+        flush(st, clean)
         a.record(st)
         L.step(graph)
         b.record(st)
@@ -497,14 +523,19 @@ def measure_workload(wl, d, dev, args, weights=None, full=False, flush=None):
     wbytes = active * weight_bytes_per_expert(wl)
     use_flush = flush if (flush is not None and wbytes < 4 * L2_BYTES) else None
     ms = time_steps(L, args.steps, True, use_flush)
+    # the same steps after a write-only flush, whose dirty lines the step
+    # itself must write back (for comparison with the usual practice)
+    ms_dirty = time_steps(L, args.steps, True, use_flush, clean=False) if use_flush is not None else None
     t_g1, t_g2 = L.time_gemms(args.steps)
     e2e_ms, e2e_bytes = time_e2e(L, args.steps, args.warmup, graph=True)
     res = {"T": wl.T, "ms_per_step": ms / args.steps, "tokens_per_s": wl.T * args.steps / (ms / 1e3),
            "active_experts": active, "launches_per_step": launches,
-           "l2": "flushed between timed steps" if use_flush is not None else
+           "l2": use_flush.describe() if use_flush is not None else
                  "not flushed: each step streams the active experts' weights (> 4x L2)",
            "e2e": {"value": wl.T * args.steps / (e2e_ms / 1e3), "unit": UNIT, **e2e_bytes,
                    "launch": "CUDA graph replay"}}
+    if ms_dirty is not None:
+        res["ms_per_step_after_write_only_flush"] = ms_dirty / args.steps
     if full:
         ms_direct = time_steps(L, args.steps, False, use_flush)
         e2e_d_ms, _ = time_e2e(L, args.steps, args.warmup, graph=False)
@@ -665,7 +696,7 @@ def measure_rope(rw, dev, args, flush):
     """The attention-side step (inverse rotary + per-head E4M3, one launch):
     tokens/s and HBM GB/s of its algorithmic bytes (x in, codes and scales
     out, positions and the table rows it reads), each step timed alone with L2
-    rewritten in between (its data fits in L2)."""
+    emptied in between (its data fits in L2)."""
     import torch
     import mixture_experts_layer_22_b200 as moe
     d = syn.rope_inputs(rw)
@@ -682,15 +713,19 @@ def measure_rope(rw, dev, args, flush):
     torch.cuda.synchronize(dev)
     if int(status.item()) != 0:
         raise SystemExit(f"{rw.name}: device status {int(status.item())}")
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    for a, b in ev:
-        with torch.cuda.stream(st):
-            flush.add_(1)
-        a.record(st)
-        moe.inv_rope_quant(s, x, pos, cs, q, sc, status, st)
-        b.record(st)
-    torch.cuda.synchronize(dev)
-    ms = sum(a.elapsed_time(b) for a, b in ev) / args.steps
+    def timed(clean):
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(args.steps)]
+        for a, b in ev:
+            flush(st, clean)
+            a.record(st)
+            moe.inv_rope_quant(s, x, pos, cs, q, sc, status, st)
+            b.record(st)
+        torch.cuda.synchronize(dev)
+        return sum(a.elapsed_time(b) for a, b in ev) / args.steps
+
+    ms = timed(True)
+    ms_dirty = timed(False)
     heads = rw.T * rw.n_heads
     nbytes = heads * rw.head_dim * 3 + heads * 4 + rw.T * 4 + rw.T * rw.rot_dim * 4
     hbm_peak = measured_peaks()[0]
@@ -699,7 +734,8 @@ def measure_rope(rw, dev, args, flush):
             "roofline": {"bound": "hbm", "achieved": nbytes / (ms * 1e-3) / 1e9, "peak": hbm_peak, "unit": "GB/s",
                          "frac": nbytes / (ms * 1e-3) / 1e9 / hbm_peak, "algorithmic_bytes": nbytes,
                          "traffic": captured_traffic(f"{rw.name} T={rw.T} rope")},
-            "l2": "flushed between timed steps", "launches_per_step": 1}
+            "ms_per_step_after_write_only_flush": ms_dirty,
+            "l2": flush.describe(), "launches_per_step": 1}
 
 
 def rope_main(args):
@@ -711,7 +747,7 @@ def rope_main(args):
         rw = rw.with_T(args.T)
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
-    flush = torch.empty(64 * 2 ** 20, dtype=torch.float32, device=dev)
+    flush = L2Flush(torch, dev)
     r = measure_rope(rw, dev, args, flush)
     line = {"metric": "inverse-RoPE + per-head E4M3 tokens/s", "value": r["tokens_per_s"], "unit": UNIT,
             "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": r["ms_per_step"],
@@ -727,7 +763,7 @@ def rope_main(args):
 def sweep(args, dev, d_head, weights_head, wl_head):
     """Every configuration besides the headline, measured the same way."""
     import torch
-    flush = torch.empty(64 * 2 ** 20, dtype=torch.float32, device=dev)     # 256 MB > L2
+    flush = L2Flush(torch, dev)
     out = {}
     cache = {"key": (wl_head.name, wl_head.wdtype, wl_head.adtype), "weights": weights_head,
              "host": {k: d_head[k] for k in ("w13", "w13_scale", "w2", "w2_scale")}}
