@@ -214,6 +214,26 @@ __device__ __forceinline__ void rope_head(const uint4 w0, const uint4 w1, const 
     }
 }
 
+// kP passes of 32 / kL heads from h00 on: this lane's two 16-byte chunks of
+// each head (zeros past h_end), all loads issued before any is used.
+template <int kL, int kP>
+__device__ __forceinline__ void load_pass(uint4 (&w)[kP][2], const __nv_bfloat16 *__restrict__ x, long long row,
+                                          int h00, int h_end, int sub, int off0, int off1)
+{
+    constexpr int kHd = 16 * kL, kHpw = 32 / kL;
+#pragma unroll
+    for (int u = 0; u < kP; ++u) {
+        const int h = h00 + u * kHpw + sub;
+        if (h < h_end) {
+            const __nv_bfloat16 *src = x + (row + h) * kHd;
+            w[u][0] = __ldg(reinterpret_cast<const uint4 *>(src + off0));
+            w[u][1] = __ldg(reinterpret_cast<const uint4 *>(src + off1));
+        } else {
+            w[u][0] = w[u][1] = make_uint4(0u, 0u, 0u, 0u);
+        }
+    }
+}
+
 // Each head is handled by kL = head_dim / 16 lanes with 16 elements per lane,
 // read as two 8-element chunks (two 16-byte loads), so that every rotary pair
 // has both its elements in one lane:
@@ -228,7 +248,10 @@ __device__ __forceinline__ void rope_head(const uint4 w0, const uint4 w1, const 
 // instructions per pack and output half; the quotient by the head's scale
 // another three per pack.  A warp processes 32 / kL heads at once and takes
 // one token and a chunk of hc of its heads per item: the token's position and
-// the lane's rotary coefficients are loaded once for the chunk.
+// the lane's rotary coefficients are loaded once for the chunk.  The loads of
+// an item overlap: the next item's position is read while this one runs, and
+// the first pass of head rows (which do not depend on the position) is
+// requested before the coefficients.
 template <int kL, bool kInterleaved>
 __global__ void __launch_bounds__(256, 2) inv_rope_quant_kernel(const __nv_bfloat16 *__restrict__ x,
                                                              const int32_t *__restrict__ positions,
@@ -248,12 +271,17 @@ __global__ void __launch_bounds__(256, 2) inv_rope_quant_kernel(const __nv_bfloa
     const long long n_items = static_cast<long long>(T) * n_chunks;
     int off0, off1, pbase, n_rot;
     lane_layout<kL, kInterleaved>(li, rot_dim, off0, off1, pbase, n_rot);
+    constexpr int kP = 4;                          // passes whose loads are in flight together
+    int p_next = warp_g < n_items ? __ldg(positions + static_cast<int>(warp_g / n_chunks)) : 0;
     for (long long item = warp_g; item < n_items; item += n_warps) {
         const int t = static_cast<int>(item / n_chunks);
         const int h_begin = static_cast<int>(item % n_chunks) * hc;
         const int h_end = min(n_heads, h_begin + hc);
-        const int p = __ldg(positions + t);
+        const int p = p_next;
+        if (item + n_warps < n_items) p_next = __ldg(positions + static_cast<int>((item + n_warps) / n_chunks));
         const long long row = static_cast<long long>(t) * n_heads;
+        uint4 w[kP][2];
+        load_pass<kL, kP>(w, x, row, h_begin, h_end, sub, off0, off1);
         if (p < 0 || p >= max_pos) {                    // the same for the whole warp
             if (lane == 0 && status) set_status(status, MOE_ERR_DEVICE_CHECK);
             for (int h = h_begin + sub; h < h_end; h += kHpw) {
@@ -266,22 +294,9 @@ __global__ void __launch_bounds__(256, 2) inv_rope_quant_kernel(const __nv_bfloa
         }
         float2 C[4], S[4], NS[4];
         load_coeffs(cos_sin + static_cast<size_t>(p) * rot_dim, pbase, half, n_rot, C, S, NS);
-        // kP passes of kHpw heads at a time: every load of the kP passes is
-        // issued before any is used (more bytes in flight per lane)
-        constexpr int kP = 4;
+        // kP passes of kHpw heads at a time (more bytes in flight per lane)
         for (int h00 = h_begin; h00 < h_end; h00 += kP * kHpw) {
-            uint4 w[kP][2];
-#pragma unroll
-            for (int u = 0; u < kP; ++u) {
-                const int h = h00 + u * kHpw + sub;
-                if (h < h_end) {
-                    const __nv_bfloat16 *src = x + (row + h) * kHd;
-                    w[u][0] = __ldg(reinterpret_cast<const uint4 *>(src + off0));
-                    w[u][1] = __ldg(reinterpret_cast<const uint4 *>(src + off1));
-                } else {
-                    w[u][0] = w[u][1] = make_uint4(0u, 0u, 0u, 0u);
-                }
-            }
+            if (h00 != h_begin) load_pass<kL, kP>(w, x, row, h00, h_end, sub, off0, off1);
 #pragma unroll
             for (int u = 0; u < kP; ++u) {
                 const int h = h00 + u * kHpw + sub;
