@@ -210,7 +210,7 @@ int moe_gather(const moe_shape_t *shape, const void *x, const int32_t *sorted_ro
  *   codes of h / a2_scale (saturated).  Only rows of segments are written.
  *   fp32 accumulation in tensor memory.  In the Swap-AB variant an expert's
  *   weight tile is streamed once per row tile of its segment: once when the
- *   segment fits one tile (256 rows, or 64 rows for E4M3 weights with bf16
+ *   segment fits one tile (256 rows, or 16 rows for E4M3 weights with bf16
  *   activations); the row tiles of one weight tile run side by side, so a
  *   repeat read comes mostly from L2.
  *   E4M3 weights with bf16 activations (this call and step 5): the
