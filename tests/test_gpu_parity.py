@@ -328,18 +328,19 @@ def test_fused_edge_cases(wl, pad):
         assert rel_err(got, ref, "bf16") <= BF16_TOL, (variant, pad)
 
 
-def _random_shapes(n=16, seed=7):
+def _random_shapes(n=16, seed=7, e_choices=(1, 2, 5, 8, 16, 33, 64), tag="rand"):
     """Seeded random layer shapes across the supported space (H, I multiples
-    of 128; ragged T; 1 to 64 experts; top-1 to top-8; softmax or sigmoid
-    gate; a shared expert or none; bf16 or E4M3 weights; both operand
-    orders).  The list is fixed by the seed, so a failure names its shape."""
+    of 128; ragged T; 1 to 64 experts, or the given counts; top-1 to top-8;
+    softmax or sigmoid gate; a shared expert or none; bf16 or E4M3 weights;
+    both operand orders).  The list is fixed by the seed, so a failure names
+    its shape."""
     rng = np.random.default_rng(seed)
     out = []
     for i in range(n):
-        E = int(rng.choice([1, 2, 5, 8, 16, 33, 64]))
+        E = int(rng.choice(e_choices))
         k = int(rng.integers(1, min(E, 8) + 1))
         w8 = bool(rng.random() < 0.25)
-        wl = syn.Workload(f"rand{i}", T=int(rng.integers(1, 700)), H=int(rng.choice([128, 256, 384, 640])),
+        wl = syn.Workload(f"{tag}{i}", T=int(rng.integers(1, 700)), H=int(rng.choice([128, 256, 384, 640])),
                           I=int(rng.choice([128, 256, 512, 896])), E=E, k=k,
                           n_shared=int(rng.random() < 0.3),
                           gate=syn.SIGMOID if rng.random() < 0.3 else syn.SOFTMAX,
@@ -351,7 +352,8 @@ def _random_shapes(n=16, seed=7):
     return out
 
 
-@pytest.mark.parametrize("wl,variant,pad", _random_shapes(),
+@pytest.mark.parametrize("wl,variant,pad",
+                         _random_shapes() + _random_shapes(12, seed=11, e_choices=(3, 24, 128, 256, 512), tag="randE"),
                          ids=lambda v: getattr(v, "name", str(v)))
 def test_fused_random_shapes(wl, variant, pad):
     d = syn.make_inputs(wl)
