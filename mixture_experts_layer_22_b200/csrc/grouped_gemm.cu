@@ -419,17 +419,14 @@ __global__ void __launch_bounds__(Cfg<kMode, kSwap, kFp8, kBN, kHiLo, kPair>::kT
     const int rem = S.n_tiles % S.G;
     // whole tiles throughout when the idle share of the last round, over
     // all rounds, is at most p.stream_k percent, or when the idle K-steps
-    // per CTA are fewer than a split would cost.  The second test also holds
-    // with fewer tiles than CTAs: a few short tiles split over every SM give
-    // each CTA a K-step or two, behind its fixed set-up and a partial-tile
-    // epilogue, and the CTAs that finish split tiles then add the partials.
+    // per CTA are fewer than a split would cost
     const int rounds = (S.n_tiles + S.G - 1) / S.G;
     const long long idle = static_cast<long long>(S.G) * rounds - S.n_tiles;
-    const bool full_enough = (S.n_tiles >= S.G && 100 * idle <= static_cast<long long>(p.stream_k) * S.G * rounds) ||
-                             idle * S.KT <= static_cast<long long>(p.split_cost) * S.G;
+    const bool full_enough = S.n_tiles >= S.G && (100 * idle <= static_cast<long long>(p.stream_k) * S.G * rounds ||
+                                                  idle * S.KT <= static_cast<long long>(p.split_cost) * S.G);
     if (!p.stream_k || rem == 0) S.dp_tiles = S.n_tiles;
-    else if (full_enough) S.dp_tiles = S.n_tiles;
     else if (S.n_tiles < S.G) S.dp_tiles = 0;
+    else if (full_enough) S.dp_tiles = S.n_tiles;
     else S.dp_tiles = (S.n_tiles / S.G - 1) * S.G;
     S.sk_tiles = S.n_tiles - S.dp_tiles;
     S.sk_total = static_cast<long long>(S.sk_tiles) * S.KT;
